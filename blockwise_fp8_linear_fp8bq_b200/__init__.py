@@ -1,0 +1,253 @@
+"""Blockwise-FP8 linear layer for NVIDIA B200 (sm_100a): thin Python binding.
+
+Every step of the computation runs in the CUDA library ``libfp8bq.so`` (C ABI
+in ``include/fp8bq.h``); this module only allocates outputs with PyTorch,
+marshals pointers and the current CUDA stream, and turns status codes into
+exceptions.  There is no CPU or PyTorch fallback: without the library, or
+without a CUDA device, every call raises.
+
+Method: "Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX 5090 within $5090"
+(section "方法"): activations quantized in 1x128 groups, weights in 128x128
+blocks, E4M3 codes with one scale per group/block (FP32, or power-of-two
+UE8M0 for the MXFP8 route), FP8 GEMMs with FP32 accumulation, BF16 output.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "Fp8bqError", "lib", "lib_path",
+    "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_weight", "Operand",
+    "row_operand", "block_operand", "bf16_operand", "gemm", "linear_forward", "linear_dgrad",
+    "linear_wgrad", "check",
+]
+
+SCALE_FP32 = 0
+SCALE_UE8M0 = 1
+GRAN_ROW = 0
+GRAN_BLOCK = 1
+_E4M3 = 0
+_BF16 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libfp8bq.so")
+_lib = None
+
+
+class Fp8bqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {_status_string(status)} ({status})")
+
+
+class _COperand(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("ld", ctypes.c_int64),
+        ("dtype", ctypes.c_int32),
+        ("k_major", ctypes.c_int32),
+        ("scales", ctypes.c_void_p),
+        ("gran", ctypes.c_int32),
+        ("fmt", ctypes.c_int32),
+        ("s_stride_k", ctypes.c_int64),
+        ("s_stride_r", ctypes.c_int64),
+    ]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libfp8bq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing; build it with "
+                              "`python -m blockwise_fp8_linear_fp8bq_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        for name in ("fp8bq_quantize_act", "fp8bq_quantize_act_t", "fp8bq_quantize_weight"):
+            f = getattr(L, name)
+            f.restype = i32
+            f.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp]
+        L.fp8bq_gemm.restype = i32
+        L.fp8bq_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
+                                 i64, i64, ctypes.c_uint32, vp]
+        L.fp8bq_row_scale_ld.restype = i64
+        L.fp8bq_row_scale_ld.argtypes = [i64]
+        L.fp8bq_scales_bytes.restype = i64
+        L.fp8bq_scales_bytes.argtypes = [i32, i32, i64, i64]
+        L.fp8bq_check.restype = i32
+        L.fp8bq_check.argtypes = [vp]
+        L.fp8bq_last_cuda_error.restype = i32
+        L.fp8bq_status_string.restype = ctypes.c_char_p
+        L.fp8bq_status_string.argtypes = [i32]
+        L.fp8bq_version.restype = i32
+        _lib = L
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().fp8bq_status_string(status).decode()
+    except Exception:  # pragma: no cover - library missing
+        return "status"
+
+
+def _raise(status: int, what: str):
+    if status != 0:
+        err = Fp8bqError(status, what)
+        if status == -5:
+            err.args = (err.args[0] + f" [cudaError {lib().fp8bq_last_cuda_error()}]",)
+        raise err
+
+
+def _stream(t: torch.Tensor) -> int:
+    if not t.is_cuda:
+        raise ValueError("fp8bq runs on CUDA tensors only (no CPU path)")
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _check_bf16(x: torch.Tensor, name: str):
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D row-major bf16 CUDA tensor")
+
+
+def row_scale_ld(rows: int) -> int:
+    """Row stride of a 1x128-group scale array (rows rounded up to 128)."""
+    return (rows + 127) // 128 * 128
+
+
+def _scale_dtype(fmt: int):
+    if fmt == SCALE_FP32:
+        return torch.float32
+    if fmt == SCALE_UE8M0:
+        return torch.uint8
+    raise ValueError("fmt must be SCALE_FP32 or SCALE_UE8M0")
+
+
+def quantize_act(x: torch.Tensor, fmt: int = SCALE_FP32):
+    """X [M,K] bf16 -> (q [M,K] float8_e4m3fn, scales [K/128, round_up(M,128)])."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty((K // 128, row_scale_ld(M)), dtype=_scale_dtype(fmt), device=x.device)
+    st = lib().fp8bq_quantize_act(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), fmt,
+                                  _stream(x))
+    _raise(st, "fp8bq_quantize_act")
+    return q, s
+
+
+def quantize_act_t(x: torch.Tensor, fmt: int = SCALE_FP32):
+    """X [M,K] bf16 -> (qt [K,M] float8_e4m3fn, scales [M/128, round_up(K,128)])."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = torch.empty((K, M), dtype=torch.float8_e4m3fn, device=x.device)
+    s = torch.empty((M // 128, row_scale_ld(K)), dtype=_scale_dtype(fmt), device=x.device)
+    st = lib().fp8bq_quantize_act_t(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), fmt,
+                                    _stream(x))
+    _raise(st, "fp8bq_quantize_act_t")
+    return q, s
+
+
+def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32):
+    """W [N,K] bf16 -> (q [N,K] float8_e4m3fn, scales [K/128, ceil(N/128)])."""
+    _check_bf16(w, "w")
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
+    s = torch.empty((K // 128, (N + 127) // 128), dtype=_scale_dtype(fmt), device=w.device)
+    st = lib().fp8bq_quantize_weight(w.data_ptr(), N, K, w.stride(0), q.data_ptr(), s.data_ptr(), fmt,
+                                     _stream(w))
+    _raise(st, "fp8bq_quantize_weight")
+    return q, s
+
+
+@dataclass
+class Operand:
+    """A GEMM operand seen as a logical [rows, C] matrix (C = contraction)."""
+    data: torch.Tensor
+    k_major: bool
+    gran: int
+    scales: Optional[torch.Tensor]
+    fmt: int
+    s_stride_k: int
+    s_stride_r: int
+    bf16: bool = False
+
+    @property
+    def rows(self) -> int:
+        return self.data.shape[0] if self.k_major else self.data.shape[1]
+
+    @property
+    def contraction(self) -> int:
+        return self.data.shape[1] if self.k_major else self.data.shape[0]
+
+    def _c(self) -> _COperand:
+        return _COperand(self.data.data_ptr(), self.data.stride(0), _BF16 if self.bf16 else _E4M3,
+                         int(self.k_major), 0 if self.scales is None else self.scales.data_ptr(),
+                         self.gran, self.fmt, self.s_stride_k, self.s_stride_r)
+
+
+def row_operand(q: torch.Tensor, scales: torch.Tensor, fmt: int) -> Operand:
+    """Codes + scales from quantize_act / quantize_act_t (1x128 row groups)."""
+    return Operand(q, True, GRAN_ROW, scales, fmt, scales.shape[1], 1)
+
+
+def block_operand(q: torch.Tensor, scales: torch.Tensor, fmt: int, transposed: bool = False) -> Operand:
+    """Codes + scales from quantize_weight.  transposed=True reads W [N,K] as W^T
+    (rows = W's columns, contraction over W's rows) without moving any data."""
+    if not transposed:
+        return Operand(q, True, GRAN_BLOCK, scales, fmt, scales.shape[1], 1)
+    return Operand(q, False, GRAN_BLOCK, scales, fmt, 1, scales.shape[1])
+
+
+def bf16_operand(x: torch.Tensor, fmt: int) -> Operand:
+    """BF16 activations to be quantized inside the GEMM (1x128 groups)."""
+    _check_bf16(x, "x")
+    return Operand(x, True, GRAN_ROW, None, fmt, 0, 1, bf16=True)
+
+
+def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """D = deq(A) . deq(B)^T in BF16 ([A.rows, B.rows])."""
+    M, N, K = A.rows, B.rows, A.contraction
+    if B.contraction != K:
+        raise ValueError("contraction mismatch")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.data.device)
+    ca, cb = A._c(), B._c()
+    st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0), 0,
+                          _stream(out))
+    _raise(st, "fp8bq_gemm")
+    return out
+
+
+def linear_forward(x: torch.Tensor, w: torch.Tensor, fmt: int = SCALE_FP32) -> torch.Tensor:
+    """Y = X W^T with X in 1x128 groups and W in 128x128 blocks."""
+    qx, sx = quantize_act(x, fmt)
+    qw, sw = quantize_weight(w, fmt)
+    return gemm(row_operand(qx, sx, fmt), block_operand(qw, sw, fmt))
+
+
+def linear_dgrad(dy: torch.Tensor, qw: torch.Tensor, sw: torch.Tensor, fmt: int = SCALE_FP32) -> torch.Tensor:
+    """dX = dY W, dY in 1x128 groups along N, W's 128x128 blocks read transposed."""
+    qd, sd = quantize_act(dy, fmt)
+    return gemm(row_operand(qd, sd, fmt), block_operand(qw, sw, fmt, transposed=True))
+
+
+def linear_wgrad(dy: torch.Tensor, x: torch.Tensor, fmt: int = SCALE_FP32) -> torch.Tensor:
+    """dW = dY^T X, both operands in 1x128 groups along the tokens."""
+    qdt, sdt = quantize_act_t(dy, fmt)
+    qxt, sxt = quantize_act_t(x, fmt)
+    return gemm(row_operand(qdt, sdt, fmt), row_operand(qxt, sxt, fmt))
+
+
+def check(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Synchronize and raise if a GEMM kernel's bounded wait expired."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    _raise(lib().fp8bq_check(s.cuda_stream), "fp8bq_check")

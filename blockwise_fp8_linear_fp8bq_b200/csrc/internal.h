@@ -1,0 +1,45 @@
+// internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace fp8bq {
+
+inline int64_t round_up128(int64_t r) { return (r + 127) / 128 * 128; }
+
+cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                             int fmt, cudaStream_t stream);
+cudaError_t launch_quant_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt,
+                               void* scales, int fmt, cudaStream_t stream);
+cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q,
+                                void* scales, int fmt, cudaStream_t stream);
+
+// A validated GEMM problem, in the library's internal form.
+struct GemmOperand {
+  const void* data;
+  int64_t ld;
+  bool bf16;     // operand A given as BF16 (quantized inside the GEMM)
+  bool k_major;  // contraction contiguous
+  const void* scales;
+  bool row_groups;  // 1x128 row groups (else 128x128 blocks)
+  int64_t s_stride_k;
+  int64_t s_stride_r;
+};
+
+struct GemmProblem {
+  GemmOperand a, b;
+  void* d;
+  int64_t M, N, K, ldd;
+  int fmt;  // kFmtFp32 / kFmtUe8m0 (both operands)
+};
+
+// Launches the GEMM; returns a cudaError_t (cudaSuccess on success).  Sets
+// *unsupported when the operand combination is not built.
+cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream, bool* unsupported);
+
+// Device status word of the GEMM kernels (0 = ok, else a timeout code).
+// Reads and clears it after synchronizing `stream`.
+cudaError_t read_and_clear_device_status(cudaStream_t stream, int* status);
+
+}  // namespace fp8bq

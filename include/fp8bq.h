@@ -1,0 +1,182 @@
+/*
+ * fp8bq.h -- C ABI of the blockwise-FP8 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The method (page titles and sections):
+ *   "Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX 5090 within $5090" (agihunt
+ *   paper digest), section "方法": Transformer linear layers are trained in
+ *   blockwise FP8 from random init, activations grouped by 128, weights in
+ *   128x128 blocks, MXFP8 on Blackwell, master weights and optimizer state kept
+ *   in BF16/FP32; section "术语", entry "blockwise FP8": one scale per local
+ *   block so that an outlier cannot blow up a single per-tensor scale.
+ *   "清华开源 Puro-2B" (ModelScope community post), section
+ *   "精度：FP8 分块量化与净效率收益": the main linear layers' matmuls run in FP8
+ *   (fine-grained block quantization in the manner of DeepSeek-V3).
+ *
+ * Conventions shared by every call:
+ *   - All data pointers are DEVICE pointers to caller-owned memory.  The library
+ *     allocates no device memory and never frees caller memory.
+ *   - Every compute call is asynchronous on `stream` (NULL = legacy default
+ *     stream) and never synchronizes; errors it can see at launch are returned
+ *     at once, errors that happen on the device surface at fp8bq_check().
+ *   - Matrices are row-major; every `ld*` is a leading dimension in ELEMENTS.
+ *   - FP8 data is OCP E4M3FN (bias 7, max 448, no infinities).  BF16 inputs
+ *     must be finite.
+ *   - Scale arrays (a library choice; the pages fix none):
+ *       1x128 row groups of an operand with R rows and contraction length C:
+ *         scales[cb * fp8bq_row_scale_ld(R) + r], cb = k / 128; the row
+ *         stride is R rounded up to a multiple of 128 and the pad entries
+ *         r >= R hold the neutral scale (1.0f, or the byte 127);
+ *       128x128 blocks of W [N,K]: scales[kb * ceil(N/128) + nb].
+ *     FP32 scales are `float`; UE8M0 scales are one byte e + 127 meaning 2^e.
+ *   - Scale definitions:  FP32: s = fl32(amax / 448) (s = 1 for an all-zero
+ *     group), code q = E4M3_RNE_satfinite(fl32(x / s)).  UE8M0: e = the least
+ *     integer with amax <= 448 * 2^e, clamped to [-127, 127] (e = 0 for an
+ *     all-zero group), q = E4M3_RNE_satfinite(x * 2^-e).
+ *   - Return value: FP8BQ_OK or one of the negative FP8BQ_ERR_* codes.  A call
+ *     that returns an error has launched nothing.
+ */
+#ifndef FP8BQ_H
+#define FP8BQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* fp8bq_stream_t;
+
+#define FP8BQ_OK 0
+#define FP8BQ_ERR_INVALID_ARG (-1) /* null pointer or unknown enum value            */
+#define FP8BQ_ERR_SHAPE (-2)       /* bad dimension (see each call)                 */
+#define FP8BQ_ERR_ALIGN (-3)       /* pointer or leading dimension not 16-B aligned */
+#define FP8BQ_ERR_UNSUPPORTED (-4) /* no sm_100 device, or an operand combination   */
+                                   /* this library does not build                   */
+#define FP8BQ_ERR_CUDA (-5)        /* a CUDA call failed; see fp8bq_last_cuda_error */
+#define FP8BQ_ERR_TIMEOUT (-6)     /* a bounded wait inside a GEMM kernel expired   */
+
+typedef enum { FP8BQ_SCALE_FP32 = 0, FP8BQ_SCALE_UE8M0 = 1 } fp8bq_scale_fmt;
+typedef enum { FP8BQ_GRAN_ROW_1x128 = 0, FP8BQ_GRAN_BLOCK_128x128 = 1 } fp8bq_gran;
+typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
+
+/*
+ * One GEMM operand, seen as a logical matrix [rows, C] whose second index runs
+ * over the contraction C.
+ *   data     E4M3 codes (dtype E4M3), or BF16 values (dtype BF16: operand A
+ *            only, quantized inside the GEMM with 1x128 groups and format
+ *            `fmt`, bit-identical to fp8bq_quantize_act).
+ *   ld       leading dimension in elements; ld * element size % 16 == 0.
+ *   k_major  1: element (r, k) is data[r*ld + k] (contraction contiguous);
+ *            0: element (r, k) is data[k*ld + r] (rows contiguous).  k_major = 0
+ *            is accepted for a 128x128-block operand B (the dgrad GEMM reads
+ *            W [N,K] as W^T this way, without a transpose pass).
+ *   scales   scale array (ignored when dtype is BF16).
+ *   gran     FP8BQ_GRAN_ROW_1x128 (A, or B in the weight-gradient GEMM) or
+ *            FP8BQ_GRAN_BLOCK_128x128 (B only).
+ *   fmt      FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0; A and B must agree.
+ *   s_stride_k, s_stride_r
+ *            the scale of element (r, k) is scales[(k/128)*s_stride_k +
+ *            t*s_stride_r], t = r (row groups) or t = r/128 (blocks).  Row
+ *            groups need s_stride_r == 1 and s_stride_k a multiple of 128;
+ *            blocks are either (ceil(rows/128), 1) or, for W^T, (1, C/128).
+ */
+typedef struct fp8bq_operand {
+  const void* data;
+  int64_t ld;
+  int32_t dtype;
+  int32_t k_major;
+  const void* scales;
+  int32_t gran;
+  int32_t fmt;
+  int64_t s_stride_k;
+  int64_t s_stride_r;
+} fp8bq_operand;
+
+/*
+ * 1x128 activation quantization ("方法": activations grouped by 128).
+ *   x       BF16 [M, K], leading dimension ldx (ldx >= K, ldx % 8 == 0).
+ *   q       E4M3 [M, K], leading dimension K.
+ *   scales  [K/128][fp8bq_row_scale_ld(M)] of float (FP32) or uint8 (UE8M0).
+ * Each row's K values form K/128 groups of 128 consecutive columns.
+ * Errors: ERR_INVALID_ARG (null pointer, bad fmt), ERR_SHAPE (M < 0, K < 0,
+ * K % 128 != 0, ldx < K), ERR_ALIGN (x, q or scales not 16-B aligned, or
+ * ldx % 8 != 0).  M == 0 or K == 0 is a no-op.
+ */
+int fp8bq_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                       int fmt, fp8bq_stream_t stream);
+
+/*
+ * 1x128 quantization along the token dimension, for the weight-gradient GEMM
+ * that contracts over tokens: the act quantizer applied to X^T.
+ *   x       BF16 [M, K], leading dimension ldx.
+ *   qt      E4M3 [K, M], leading dimension M (the transpose of the codes).
+ *   scales  [M/128][fp8bq_row_scale_ld(K)].
+ * Errors: as fp8bq_quantize_act, with ERR_SHAPE when M % 128 != 0 (M is the
+ * contraction here) and ERR_ALIGN when K % 8 != 0 or ldx % 8 != 0.
+ */
+int fp8bq_quantize_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt, void* scales,
+                         int fmt, fp8bq_stream_t stream);
+
+/*
+ * 128x128 weight-block quantization ("方法": weights in 128x128 blocks).
+ *   w       BF16 [N, K], leading dimension ldw (ldw >= K, ldw % 8 == 0).
+ *   q       E4M3 [N, K], leading dimension K.
+ *   scales  [K/128][ceil(N/128)].  A block at the edge (N % 128 != 0) covers
+ *           only its valid rows.
+ * Errors: ERR_SHAPE when K % 128 != 0; otherwise as fp8bq_quantize_act.
+ */
+int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, void* scales,
+                          int fmt, fp8bq_stream_t stream);
+
+/*
+ * Blockwise-FP8 GEMM ("精度" section of the ModelScope post; "方法" of the
+ * digest):  D[m, n] = sum over 128-blocks kb of  sA(m,kb) * sB(n,kb) *
+ * sum_{k in kb} qA[m,k] * qB[n,k], accumulated in FP32 on the tensor cores,
+ * rounded once to BF16 (round-to-nearest-even).
+ *   forward  A = quantize_act(X), B = quantize_weight(W)        D = Y [M, N]
+ *   dgrad    A = quantize_act(dY), B = W^T (k_major = 0)        D = dX [M, K_w]
+ *   wgrad    A = quantize_act_t(dY), B = quantize_act_t(X)      D = dW [N, K]
+ * FP32 scales run the per-128-K promotion path (partial products in tensor
+ * memory, rescaled into FP32 accumulators); UE8M0 scales run the block-scaled
+ * MMA (MXFP8 route).
+ *   D       BF16 [M, N], leading dimension ldd (ldd >= N, ldd % 8 == 0).
+ *   K       contraction length, K % 128 == 0, K > 0.
+ *   flags   0 (reserved for future hints; other values give ERR_INVALID_ARG).
+ * Errors: ERR_INVALID_ARG, ERR_SHAPE (M,N <= 0, K % 128 != 0, N % 8 != 0),
+ * ERR_ALIGN (a pointer not 16-B aligned, a leading dimension not a multiple
+ * of 16 bytes), ERR_UNSUPPORTED (mixed scale formats, BF16 B, row-group B
+ * that is not k-major), ERR_CUDA (tensor-map encoding or launch failed).
+ */
+int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
+               int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream);
+
+/* Row stride of a 1x128-group scale array: rows rounded up to 128. */
+int64_t fp8bq_row_scale_ld(int64_t rows);
+
+/* Bytes of the scale array for an operand with `rows` rows and contraction
+ * `contraction` (a multiple of 128); -1 on bad arguments. */
+int64_t fp8bq_scales_bytes(int gran, int fmt, int64_t rows, int64_t contraction);
+
+/*
+ * Synchronizes `stream`, then reports the first device-side failure since the
+ * last check: FP8BQ_ERR_TIMEOUT if a GEMM kernel's bounded wait expired (the
+ * kernel then stopped early and its output is undefined), FP8BQ_ERR_CUDA if
+ * the stream reported an error.  Clears the recorded state.
+ */
+int fp8bq_check(fp8bq_stream_t stream);
+
+/* The cudaError_t value behind the last FP8BQ_ERR_CUDA of this thread. */
+int fp8bq_last_cuda_error(void);
+
+/* Static text for a status code. */
+const char* fp8bq_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int fp8bq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8BQ_H */

@@ -1,0 +1,121 @@
+"""The C-ABI boundary on the CPU: libfp8bq.so loads, exports every function
+include/fp8bq.h declares, and rejects bad arguments with the documented status
+codes before it touches a device (fake pointers are never dereferenced)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA, TIMEOUT = 0, -1, -2, -3, -4, -5, -6
+P = 1 << 20  # a 16-byte aligned fake device address (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from blockwise_fp8_linear_fp8bq_b200 import build
+    build.build()
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    return fp.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp8bq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8bq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function(L):
+    names = declared_functions()
+    assert "fp8bq_gemm" in names and "fp8bq_quantize_act_t" in names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    for code in (OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA, TIMEOUT):
+        s = L.fp8bq_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert L.fp8bq_status_string(-99).decode() == "unknown status"
+    assert L.fp8bq_version() >= 100
+
+
+def test_scale_size_helpers(L):
+    assert L.fp8bq_row_scale_ld(1) == 128
+    assert L.fp8bq_row_scale_ld(256) == 256
+    assert L.fp8bq_row_scale_ld(16384) == 16384
+    # [K/128][round_up(M,128)] fp32
+    assert L.fp8bq_scales_bytes(0, 0, 200, 512) == 4 * 256 * 4
+    assert L.fp8bq_scales_bytes(0, 1, 200, 512) == 4 * 256
+    # [K/128][ceil(N/128)]
+    assert L.fp8bq_scales_bytes(1, 0, 320, 384) == 3 * 3 * 4
+    assert L.fp8bq_scales_bytes(1, 1, 151936, 2048) == 16 * 1187
+    assert L.fp8bq_scales_bytes(0, 0, 10, 100) == -1
+    assert L.fp8bq_scales_bytes(7, 0, 10, 128) == -1
+    assert L.fp8bq_scales_bytes(0, 9, 10, 128) == -1
+
+
+@pytest.mark.parametrize("fn", ["fp8bq_quantize_act", "fp8bq_quantize_act_t", "fp8bq_quantize_weight"])
+def test_quantizer_argument_checks(L, fn):
+    f = getattr(L, fn)
+    assert f(None, 128, 128, 128, P, P, 0, None) == INVALID
+    assert f(P, 128, 128, 128, None, P, 0, None) == INVALID
+    assert f(P, 128, 128, 128, P, None, 0, None) == INVALID
+    assert f(P, 128, 128, 128, P, P, 2, None) == INVALID
+    assert f(P, -1, 128, 128, P, P, 0, None) == SHAPE
+    assert f(P, 128, 128, 64, P, P, 0, None) == SHAPE        # ld < cols
+    assert f(P + 8, 128, 128, 128, P, P, 0, None) == ALIGN
+    assert f(P, 128, 128, 128, P + 4, P, 0, None) == ALIGN
+    assert f(P, 128, 128, 128, P, P + 2, 0, None) == ALIGN
+    assert f(P, 128, 128, 132, P, P, 0, None) == ALIGN       # ld % 8
+    if fn == "fp8bq_quantize_act_t":
+        assert f(P, 100, 128, 128, P, P, 0, None) == SHAPE   # tokens % 128
+        assert f(P, 128, 100, 104, P, P, 0, None) == ALIGN   # K % 8
+        assert f(P, 0, 64, 64, P, P, 0, None) == OK          # empty: no launch
+    else:
+        assert f(P, 128, 100, 128, P, P, 0, None) == SHAPE   # contraction % 128
+        assert f(P, 0, 128, 128, P, P, 0, None) == OK        # empty: no launch
+        assert f(P, 5, 0, 0, P, P, 0, None) == OK
+
+
+def _op(L, **kw):
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    d = dict(data=P, ld=512, dtype=0, k_major=1, scales=P, gran=0, fmt=0, s_stride_k=256, s_stride_r=1)
+    d.update(kw)
+    return fp._COperand(**d)
+
+
+def test_gemm_argument_checks(L):
+    M, N, K = 256, 256, 512
+    A = _op(L)
+    B = _op(L, gran=1, s_stride_k=2, s_stride_r=1)
+    g = lambda A_, B_, D=P, m=M, n=N, k=K, ldd=N, flags=0: L.fp8bq_gemm(
+        ctypes.byref(A_) if A_ is not None else None, ctypes.byref(B_) if B_ is not None else None,
+        D, m, n, k, ldd, flags, None)
+    assert g(None, B) == INVALID
+    assert g(A, None) == INVALID
+    assert g(A, B, D=None) == INVALID
+    assert g(A, B, flags=1) == INVALID
+    assert g(A, B, k=100) == SHAPE
+    assert g(A, B, n=100, ldd=104) == SHAPE          # N % 8
+    assert g(A, B, m=0) == SHAPE
+    assert g(A, B, ldd=128) == SHAPE
+    assert g(A, B, D=P + 8) == ALIGN
+    assert g(A, B, ldd=260) == ALIGN
+    assert g(_op(L, data=P + 1), B) == ALIGN
+    assert g(_op(L, ld=520), B) == ALIGN             # ld * 1 byte % 16
+    assert g(_op(L, ld=100), B) == SHAPE or g(_op(L, ld=100), B) == ALIGN
+    assert g(_op(L, scales=P + 4), B) == ALIGN
+    assert g(_op(L, scales=None), B) == INVALID
+    assert g(_op(L, s_stride_k=200), B) == SHAPE     # row-group stride % 128
+    assert g(_op(L, s_stride_r=2), B) == SHAPE
+    assert g(_op(L, dtype=5), B) == INVALID
+    assert g(_op(L, gran=3), B) == INVALID
+    assert g(_op(L, fmt=1), B) == UNSUPPORTED or g(_op(L, fmt=1), B) == INVALID  # mixed formats
+    assert g(A, _op(L, gran=1, s_stride_k=1, s_stride_r=1, fmt=1)) == UNSUPPORTED
+    assert g(_op(L, gran=1, s_stride_k=4, s_stride_r=1), B) == UNSUPPORTED  # block-scaled A
+    assert g(A, _op(L, k_major=0, ld=256)) == UNSUPPORTED   # row-group B must be k-major
+    assert g(A, _op(L, gran=1, s_stride_k=3, s_stride_r=3)) == SHAPE  # neither layout
+    assert g(A, _op(L, dtype=1, scales=0, ld=512)) == UNSUPPORTED      # BF16 B

@@ -1,0 +1,119 @@
+"""GPU parity of the three quantizers: codes and scales must equal the oracle's
+bit for bit (FP32 and UE8M0 scales), on small ragged shapes, planted special
+groups, and the full-size tensors of the synthetic Qwen3-1.7B-shaped layers."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import blockwise_fp8_linear_fp8bq_b200 as fp
+from blockwise_fp8_linear_fp8bq_b200 import synth
+from gpu_util import bits, scale_bytes, u8
+
+pytestmark = pytest.mark.gpu
+
+FMTS = [fp.SCALE_FP32, fp.SCALE_UE8M0]
+
+
+def check_act(x, fmt):
+    q, s = fp.quantize_act(x, fmt)
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_act(bits(x), fmt)
+    assert np.array_equal(u8(q), qo)
+    assert np.array_equal(scale_bytes(s), so.view(np.uint8).reshape(so.shape[0], -1))
+
+
+def check_act_t(x, fmt):
+    q, s = fp.quantize_act_t(x, fmt)
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_act_t(bits(x), fmt)
+    assert np.array_equal(u8(q), qo)
+    assert np.array_equal(scale_bytes(s), so.view(np.uint8).reshape(so.shape[0], -1))
+
+
+def check_weight(w, fmt):
+    q, s = fp.quantize_weight(w, fmt)
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_weight(bits(w), fmt)
+    assert np.array_equal(u8(q), qo)
+    assert np.array_equal(scale_bytes(s), so.view(np.uint8).reshape(so.shape[0], -1))
+
+
+def planted(x: torch.Tensor) -> torch.Tensor:
+    """Zero, constant, tiny (fp32-subnormal scale) and huge groups, signed zeros."""
+    x = x.clone()
+    x[0, :128] = 0
+    x[1, :128] = -3.25
+    x[2, :128] *= 1e-38
+    x[3, :128] *= 1e30
+    x[4, 128:256] = 0
+    x[4, 133] = -0.0
+    x[5, :] *= 2.0 ** -120
+    return x
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(256, 512), (200, 384), (1, 128), (129, 256), (64, 1024)])
+def test_quantize_act_small(fmt, shape):
+    x = synth.activations_bf16(*shape, seed=11, device="cuda")
+    if shape[0] >= 6 and shape[1] >= 256:
+        x = planted(x)
+    check_act(x, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(256, 200), (128, 8), (384, 512), (256, 136)])
+def test_quantize_act_t_small(fmt, shape):
+    x = synth.activations_bf16(*shape, seed=12, device="cuda")
+    x = x.clone()
+    x[:, 0] = 0
+    x[:128, 1] = -7.5
+    x[:, 2] *= 1e-38
+    check_act_t(x, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(512, 512), (320, 384), (1, 128), (130, 256)])
+def test_quantize_weight_small(fmt, shape):
+    w = synth.weights_bf16(*shape, seed=13, device="cuda").clone()
+    w[:128, :128] = 0
+    if shape[0] > 128:
+        w[128:, :128] *= 1e-36
+    check_weight(w, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_act_strided_input(fmt):
+    big = synth.activations_bf16(300, 640, seed=14, device="cuda")
+    x = big[:, :512]  # leading dimension 640
+    q, s = fp.quantize_act(x, fmt)
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_act(bits(x.contiguous()), fmt)
+    assert np.array_equal(u8(q), qo)
+    assert np.array_equal(scale_bytes(s), so.view(np.uint8).reshape(so.shape[0], -1))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_full_size_gate_up_operands(fmt):
+    """X[16384,2048] (act), W_gu[12288,2048] (weight), X^T (act_t)."""
+    lin = synth.GATE_UP
+    x = lin.x(3000, device="cuda")
+    check_act(x, fmt)
+    check_act_t(x, fmt)
+    check_weight(lin.w(3000, device="cuda"), fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_full_size_down_and_grads(fmt):
+    """H[16384,6144] (act), W_d[2048,6144] (weight), dY_d[16384,2048] (act + act_t)."""
+    lin = synth.DOWN
+    check_act(lin.x(3100, device="cuda"), fmt)
+    check_weight(lin.w(3100, device="cuda"), fmt)
+    dy = lin.dy(3100, device="cuda")
+    check_act(dy, fmt)
+    check_act_t(dy, fmt)
+
+
+def test_full_size_lm_head_weight():
+    w = synth.weights_bf16(synth.VOCAB, synth.HIDDEN, seed=3201, device="cuda")
+    check_weight(w, fp.SCALE_FP32)
