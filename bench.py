@@ -1,0 +1,571 @@
+"""Benchmark of the blockwise-FP8 linear layer on B200.
+
+One step = the full hot path over one batch: the four linears of one
+Qwen3-1.7B-like transformer layer (QKV 2048->4096, O 2048->2048, gate/up
+2048->12288, down 6144->2048) at M = 16384 tokens, each with
+  forward  quantize_act(X), quantize_weight(W), GEMM  Y  = X W^T
+  dgrad    quantize_act(dY),                    GEMM dX = dY W   (W^T read in place)
+  wgrad    quantize_act_t(dY), quantize_act_t(X), GEMM dW = dY^T X
+i.e. 20 quantizer and 12 GEMM launches, 4.948 TFLOP of blockwise-FP8 GEMM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--scale fp32|ue8m0]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Metric: blockwise-FP8 GEMM TFLOP/s of the whole step (GEMM FLOPs / step time
+including the quantizers), with the GEMM kernel's roofline (TFLOP/s vs the
+FP8 dense peak) and the quantizers' GB/s vs HBM in the same JSON line.
+Inputs are synthetic (seeded), resident in HBM for `value`; `e2e` repeats the
+step with the inputs copied from pinned host memory and the outputs copied
+back inside the timed region.  Multi-GPU: one process per GPU, each a replica
+on its own token batch (data-parallel shards, no collective on the data
+path): weak scaling, value summed over ranks, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from blockwise_fp8_linear_fp8bq_b200 import synth  # noqa: E402
+
+M_TOKENS = 16384
+METRIC = "blockwise-FP8 GEMM TFLOP/s & % FP8 peak; quantizer GB/s & % HBM (1 B200)"
+WORKLOAD = ("qwen3-1.7b layer linears (qkv 2048x4096, o 2048x2048, gate_up 2048x12288, "
+            "down 6144x2048) fwd+dgrad+wgrad, M=16384 tokens")
+FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+
+
+def linears(M=M_TOKENS):
+    return synth.layer_linears(M)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks --
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons sampled through NVML every
+    5 ms in a background thread while the timed region runs.  Read-only: it
+    changes no GPU setting."""
+
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
+
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []
+        self.reasons = set()
+        self.ok = False
+
+    def start(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            p = torch.cuda.get_device_properties(self.device)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            self.h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+            return
+        self.stop_flag = threading.Event()
+
+        def loop():
+            nv = self.nv
+            masks = [(n, getattr(nv, c, 0)) for n, c in self.REASONS]
+            while not self.stop_flag.is_set():
+                try:
+                    self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    for n, m in masks:
+                        if m and (r & m):
+                            self.reasons.add(n)
+                except Exception:
+                    pass
+                self.stop_flag.wait(0.005)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if not self.ok:
+            return None
+        self.stop_flag.set()
+        self.thread.join()
+        if not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(self.samples), "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------------- ours --
+class LayerStep:
+    """Device buffers and the launch sequence of one step."""
+
+    def __init__(self, fp, fmt, seed, device, only=None):
+        self.fp = fp
+        self.fmt = fmt
+        self.items = []
+        sdt = torch.float32 if fmt == fp.SCALE_FP32 else torch.uint8
+        e4 = torch.float8_e4m3fn
+        for i, lin in enumerate(linears()):
+            if only is not None and lin.name not in only:
+                continue
+            M, K, N = lin.M, lin.K, lin.N
+            s = seed + 100 * i
+            it = dict(lin=lin,
+                      x=lin.x(s, device=device), w=lin.w(s, device=device), dy=lin.dy(s, device=device),
+                      qx=torch.empty(M, K, dtype=e4, device=device),
+                      sx=torch.empty(K // 128, fp.row_scale_ld(M), dtype=sdt, device=device),
+                      qw=torch.empty(N, K, dtype=e4, device=device),
+                      sw=torch.empty(K // 128, (N + 127) // 128, dtype=sdt, device=device),
+                      qd=torch.empty(M, N, dtype=e4, device=device),
+                      sd=torch.empty(N // 128, fp.row_scale_ld(M), dtype=sdt, device=device),
+                      qdt=torch.empty(N, M, dtype=e4, device=device),
+                      sdt=torch.empty(M // 128, fp.row_scale_ld(N), dtype=sdt, device=device),
+                      qxt=torch.empty(K, M, dtype=e4, device=device),
+                      sxt=torch.empty(M // 128, fp.row_scale_ld(K), dtype=sdt, device=device),
+                      y=torch.empty(M, N, dtype=torch.bfloat16, device=device),
+                      dx=torch.empty(M, K, dtype=torch.bfloat16, device=device),
+                      dw=torch.empty(N, K, dtype=torch.bfloat16, device=device))
+            self.items.append(it)
+
+    # algorithmic bytes of each quantizer launch (bf16 read, e4m3 write, scales)
+    def quant_bytes(self):
+        sb = 4 if self.fmt == self.fp.SCALE_FP32 else 1
+        tot = 0
+        for it in self.items:
+            lin = it["lin"]
+            M, K, N = lin.M, lin.K, lin.N
+            tot += M * K * 3 + (K // 128) * M * sb          # act(X)
+            tot += N * K * 3 + (K // 128) * ((N + 127) // 128) * sb  # weight(W)
+            tot += M * N * 3 + (N // 128) * M * sb          # act(dY)
+            tot += M * N * 3 + (M // 128) * N * sb          # act_t(dY)
+            tot += M * K * 3 + (M // 128) * K * sb          # act_t(X)
+        return tot
+
+    def gemm_flops(self):
+        return sum(3 * it["lin"].flops for it in self.items)
+
+    def launches(self):
+        return 8 * len(self.items)
+
+    def run(self, ev=None):
+        """Issue the step on the current stream.  With `ev` (a list), record a
+        CUDA event pair around every launch: ev.append((kind, start, end))."""
+        fp, f = self.fp, self.fmt
+
+        def timed(kind, fn):
+            if ev is None:
+                fn()
+                return
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ev.append((kind, a, b))
+
+        for it in self.items:
+            timed("quant", lambda: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
+            timed("quant", lambda: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
+            timed("gemm", lambda: fp.gemm(fp.row_operand(it["qx"], it["sx"], f),
+                                          fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+            timed("quant", lambda: fp.quantize_act(it["dy"], f, it["qd"], it["sd"]))
+            timed("gemm", lambda: fp.gemm(fp.row_operand(it["qd"], it["sd"], f),
+                                          fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
+            timed("quant", lambda: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
+            timed("quant", lambda: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
+            timed("gemm", lambda: fp.gemm(fp.row_operand(it["qdt"], it["sdt"], f),
+                                          fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+
+
+def l2_flush(buf):
+    buf.zero_()
+
+
+def run_ours(args, rank, world, dist):
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    fp.lib()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
+    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+
+    for _ in range(args.warmup):
+        step.run()
+    fp.check()
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_events = []
+    kernel_events = []
+    for _ in range(args.steps):
+        l2_flush(flush)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        step.run(kernel_events)
+        b.record()
+        step_events.append((a, b))
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+    fp.check()
+
+    step_ms = sum(a.elapsed_time(b) for a, b in step_events)
+    gemm_ms = sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "gemm")
+    quant_ms = sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "quant")
+
+    # end to end: inputs from pinned host memory, outputs back to pinned host
+    e2e = None
+    if not args.no_e2e:
+        host_in, host_out = [], []
+        for it in step.items:
+            for k in ("x", "w", "dy"):
+                host_in.append((torch.empty_like(it[k], device="cpu").pin_memory(), it[k]))
+            for k in ("y", "dx", "dw"):
+                host_out.append((it[k], torch.empty_like(it[k], device="cpu").pin_memory()))
+        for h, d in host_in:
+            h.copy_(d)
+        bi = sum(h.numel() * h.element_size() for h, _ in host_in)
+        bo = sum(h.numel() * h.element_size() for _, h in host_out)
+        e2e_steps = max(1, min(args.steps, 5))
+        for _ in range(1):  # warm-up of the copy path
+            for h, d in host_in:
+                d.copy_(h, non_blocking=True)
+            step.run()
+            for d, h in host_out:
+                h.copy_(d, non_blocking=True)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(e2e_steps):
+            for h, d in host_in:
+                d.copy_(h, non_blocking=True)
+            step.run()
+            for d, h in host_out:
+                h.copy_(d, non_blocking=True)
+        t1.record()
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        e2e_ms = t0.elapsed_time(t1) / e2e_steps
+        fp.check()
+        e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps}
+
+    return dict(step_ms=step_ms, gemm_ms=gemm_ms, quant_ms=quant_ms, clocks=clocks, e2e=e2e,
+                flops=step.gemm_flops(), qbytes=step.quant_bytes(), launches=step.launches() * args.steps,
+                gemm_launches=len([1 for k, _, _ in kernel_events if k == "gemm"]),
+                quant_launches=len([1 for k, _, _ in kernel_events if k == "quant"]))
+
+
+# --------------------------------------------------------- oracle on CPU --
+def oracle_sample(seconds_hint: float = 10.0):
+    """Time the CPU oracle on a bounded sample of the step and extrapolate to
+    the whole step: quantizers on 256-row slabs of each tensor, GEMMs on whole
+    output rows (T rows of each of the 12 GEMMs, T = oracle threads)."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    T = oracle.num_threads()
+    rows_per_gemm = max(1, T)
+    q_elems = q_time = 0.0
+    g_flops = g_time = 0.0
+    full_q_elems = 0
+    full_flops = 0
+    for i, lin in enumerate(linears()):
+        M, K, N = lin.M, lin.K, lin.N
+        s = 7000 + 100 * i
+        slab = 256
+        x = synth.bf16_bits(synth.activations_bf16(slab, K, s))
+        w = synth.bf16_bits(synth.weights_bf16(min(N, slab), K, s + 1))
+        dy = synth.bf16_bits(synth.grads_bf16(slab, N, s + 2))
+        t = time.perf_counter()
+        qx, sx = oracle.quantize_act(x)
+        qw, sw = oracle.quantize_weight(w)
+        qd, sd = oracle.quantize_act(dy)
+        qdt, sdt = oracle.quantize_act_t(dy)
+        qxt, sxt = oracle.quantize_act_t(x)
+        q_time += time.perf_counter() - t
+        q_elems += 2 * x.size + w.size + 2 * dy.size
+        full_q_elems += 2 * M * K + N * K + 2 * M * N
+        # GEMMs: T full output rows of each, operands sized to the real contraction
+        xa = synth.bf16_bits(synth.activations_bf16(rows_per_gemm, K, s + 3))
+        qa, sa = oracle.quantize_act(xa)
+        A = oracle.row_operand(qa, sa, 0)
+        B = oracle.block_operand(*oracle.quantize_weight(synth.bf16_bits(synth.weights_bf16(N, K, s + 4))), 0)
+        t = time.perf_counter()
+        oracle.gemm(A, B)
+        g_time += time.perf_counter() - t
+        g_flops += 2.0 * rows_per_gemm * N * K
+        full_flops += 3 * lin.flops
+    # dgrad and wgrad rows cost the same per FLOP as forward rows in the oracle
+    # (one dequantized multiply-add per term), so the forward sample stands for all three
+    step_s = full_q_elems * (q_time / q_elems) + full_flops * (g_time / g_flops)
+    sample = (f"4 linears: 256-row slabs through the 3 quantizers and {rows_per_gemm} full output rows "
+              f"of each forward GEMM; {q_elems / 1e6:.1f} M quantized elements in {q_time:.2f} s, "
+              f"{g_flops / 1e9:.2f} GFLOP in {g_time:.2f} s; extrapolated to the full step")
+    return {"step_s": step_s, "tflops": full_flops / step_s / 1e12, "cores": T, "sample": sample,
+            "sample_s": q_time + g_time}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    steps = []
+    t_all = time.perf_counter()
+    res = None
+    for i in range(args.warmup + args.steps):
+        res = oracle_sample()
+        if i >= args.warmup:
+            steps.append(res["step_s"])
+    step_s = statistics.median(steps) if steps else res["step_s"]
+    flops = sum(3 * lin.flops for lin in linears())
+    value = flops / step_s / 1e12
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "scale_format": args.scale, "tokens": M_TOKENS,
+                   "parallelism": f"replicas{world}"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": time.perf_counter() - t_all,
+    }
+    print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------ kernel cases --
+def case_launchers(step, fp):
+    """name -> (kind, algorithmic units, fn) for every launch of the step; units
+    are FLOPs for GEMMs and bytes for quantizers."""
+    f = fp.SCALE_FP32 if step.fmt == fp.SCALE_FP32 else fp.SCALE_UE8M0
+    sb = 4 if f == fp.SCALE_FP32 else 1
+    out = {}
+    for it in step.items:
+        lin = it["lin"]
+        M, K, N, n = lin.M, lin.K, lin.N, lin.name
+        out[f"quant_act:x:{n}"] = ("quant", M * K * 3 + (K // 128) * M * sb,
+                                   lambda it=it: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
+        out[f"quant_weight:{n}"] = ("quant", N * K * 3 + (K // 128) * ((N + 127) // 128) * sb,
+                                    lambda it=it: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
+        out[f"quant_act:dy:{n}"] = ("quant", M * N * 3 + (N // 128) * M * sb,
+                                    lambda it=it: fp.quantize_act(it["dy"], f, it["qd"], it["sd"]))
+        out[f"quant_act_t:dy:{n}"] = ("quant", M * N * 3 + (M // 128) * N * sb,
+                                      lambda it=it: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
+        out[f"quant_act_t:x:{n}"] = ("quant", M * K * 3 + (M // 128) * K * sb,
+                                     lambda it=it: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
+        out[f"gemm_fwd:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.row_operand(it["qx"], it["sx"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+        out[f"gemm_dgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.row_operand(it["qd"], it["sd"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
+        out[f"gemm_wgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+    return out
+
+
+def run_case(args):
+    """Time single kernels of the step (L2 flushed before every launch).
+    --case all prints one line per kernel; --case NAME runs only that kernel
+    (warm-up + steps launches), e.g. for an ncu capture of one kernel."""
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    fp.lib()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
+    only = None if args.case == "all" else {args.case.split(":")[-1]}
+    step = LayerStep(fp, fmt, seed=1000, device=dev, only=only)
+    step.run()  # produce every operand once
+    torch.cuda.synchronize()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    cases = case_launchers(step, fp)
+    names = list(cases) if args.case == "all" else [args.case]
+    peaks = measured_peaks()
+    rows = []
+    for name in names:
+        if name not in cases:
+            raise SystemExit(f"unknown case {name}; one of: {', '.join(cases)}")
+        kind, units, fn = cases[name]
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            l2_flush(flush)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        fp.check()
+        ms = statistics.median(ts)
+        if kind == "gemm":
+            rate = units / (ms * 1e-3) / 1e12
+            rows.append({"case": name, "us": ms * 1e3, "tflops": rate,
+                         "frac_fp8_burst": rate / (peaks["bf16"] * FP8_OVER_BF16),
+                         "frac_nominal_4500": rate / 4500.0})
+        else:
+            rate = units / (ms * 1e-3) / 1e9
+            rows.append({"case": name, "us": ms * 1e3, "gbs": rate, "frac_hbm": rate / peaks["hbm_gbs"]})
+    for r in rows:
+        print(json.dumps(r), flush=True)
+
+
+# -------------------------------------------------------------------- main --
+def reduce_max(x: float, dist) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--scale", choices=["fp32", "ue8m0"], default="fp32")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="time single kernels instead of the step: 'all' or a name such as gemm_fwd:gate_up")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.case:
+        run_case(args)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as td
+        from datetime import timedelta
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        td.init_process_group(backend, timeout=timedelta(seconds=120))
+        dist = td
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    r = run_ours(args, rank, world, dist)
+    step_ms = reduce_max(r["step_ms"], dist) / args.steps
+    gemm_ms = reduce_max(r["gemm_ms"], dist)
+    quant_ms = reduce_max(r["quant_ms"], dist)
+    e2e_ms = reduce_max(r["e2e"]["ms_per_step"], dist) if r["e2e"] else None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample()
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = measured_peaks()
+    fp8_peak = peaks["bf16_sustained"] * FP8_OVER_BF16
+    flops = r["flops"]
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    gemm_tflops = flops * args.steps / (gemm_ms * 1e-3) / 1e12
+    quant_gbs = r["qbytes"] * args.steps / (quant_ms * 1e-3) / 1e9
+    traffic = load_traffic()
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "scale_format": args.scale, "tokens": M_TOKENS,
+                   "parallelism": f"replicas{world}", "l2": "flushed between steps (write of 2x L2)"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / fp8_peak, "traffic": traffic,
+                     "kernel": "gemm_kernel (all 12 GEMM launches of the step)",
+                     "peak_note": f"{peaks['source']} bf16 sustained x {FP8_OVER_BF16:g} (nominal FP8/BF16)"},
+        "quantizers": {"achieved_gbs": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
+                       "frac": quant_gbs / peaks["hbm_gbs"], "ms_per_step": quant_ms / args.steps,
+                       "launches_per_step": r["quant_launches"] // args.steps},
+        "gemm": {"tflops": gemm_tflops, "ms_per_step": gemm_ms / args.steps,
+                 "frac_of_nominal_4500": gemm_tflops / 4500.0,
+                 "launches_per_step": r["gemm_launches"] // args.steps},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if r["e2e"]:
+        out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
+                      "d2h_bytes_per_step": r["e2e"]["d2h_bytes_per_step"], "ms_per_step": e2e_ms}
+    if cpu is not None:
+        out["cpu_baseline"] = {"value": cpu["tflops"], "unit": "TFLOP/s", "cores": cpu["cores"],
+                               "kind": "oracle", "sample": cpu["sample"]}
+    print(json.dumps(out), flush=True)
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "blockwise_fp8_linear_fp8bq_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.startswith("gemm") or name.endswith(".cuh"):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary; null when the
+    GEMM source changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        if t.get("gemm_source_hash") != kernel_source_hash():
+            return None
+        return t.get("gemm_bytes_per_launch")
+    except Exception:
+        return None
+
+
+if __name__ == "__main__":
+    main()

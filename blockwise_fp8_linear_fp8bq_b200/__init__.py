@@ -132,36 +132,44 @@ def _scale_dtype(fmt: int):
     raise ValueError("fmt must be SCALE_FP32 or SCALE_UE8M0")
 
 
-def quantize_act(x: torch.Tensor, fmt: int = SCALE_FP32):
+def _out(buf, shape, dtype, device):
+    if buf is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    if tuple(buf.shape) != tuple(shape) or buf.dtype != dtype or not buf.is_contiguous():
+        raise ValueError(f"output buffer must be a contiguous {dtype} tensor of shape {shape}")
+    return buf
+
+
+def quantize_act(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     """X [M,K] bf16 -> (q [M,K] float8_e4m3fn, scales [K/128, round_up(M,128)])."""
     _check_bf16(x, "x")
     M, K = x.shape
-    q = torch.empty((M, K), dtype=torch.float8_e4m3fn, device=x.device)
-    s = torch.empty((K // 128, row_scale_ld(M)), dtype=_scale_dtype(fmt), device=x.device)
+    q = _out(q, (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(s, (K // 128, row_scale_ld(M)), _scale_dtype(fmt), x.device)
     st = lib().fp8bq_quantize_act(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), fmt,
                                   _stream(x))
     _raise(st, "fp8bq_quantize_act")
     return q, s
 
 
-def quantize_act_t(x: torch.Tensor, fmt: int = SCALE_FP32):
+def quantize_act_t(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     """X [M,K] bf16 -> (qt [K,M] float8_e4m3fn, scales [M/128, round_up(K,128)])."""
     _check_bf16(x, "x")
     M, K = x.shape
-    q = torch.empty((K, M), dtype=torch.float8_e4m3fn, device=x.device)
-    s = torch.empty((M // 128, row_scale_ld(K)), dtype=_scale_dtype(fmt), device=x.device)
+    q = _out(q, (K, M), torch.float8_e4m3fn, x.device)
+    s = _out(s, (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device)
     st = lib().fp8bq_quantize_act_t(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), fmt,
                                     _stream(x))
     _raise(st, "fp8bq_quantize_act_t")
     return q, s
 
 
-def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32):
+def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     """W [N,K] bf16 -> (q [N,K] float8_e4m3fn, scales [K/128, ceil(N/128)])."""
     _check_bf16(w, "w")
     N, K = w.shape
-    q = torch.empty((N, K), dtype=torch.float8_e4m3fn, device=w.device)
-    s = torch.empty((K // 128, (N + 127) // 128), dtype=_scale_dtype(fmt), device=w.device)
+    q = _out(q, (N, K), torch.float8_e4m3fn, w.device)
+    s = _out(s, (K // 128, (N + 127) // 128), _scale_dtype(fmt), w.device)
     st = lib().fp8bq_quantize_weight(w.data_ptr(), N, K, w.stride(0), q.data_ptr(), s.data_ptr(), fmt,
                                      _stream(w))
     _raise(st, "fp8bq_quantize_weight")
@@ -218,8 +226,9 @@ def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None) -> torch.Te
     M, N, K = A.rows, B.rows, A.contraction
     if B.contraction != K:
         raise ValueError("contraction mismatch")
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.data.device)
+    out = _out(out, (M, N), torch.bfloat16, A.data.device) if out is None else out
+    if out.dtype != torch.bfloat16 or out.dim() != 2 or out.stride(1) != 1 or tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be a row-major bf16 tensor of shape {(M, N)}")
     ca, cb = A._c(), B._c()
     st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0), 0,
                           _stream(out))
