@@ -8,22 +8,27 @@
 // 128x128 weight blocks, MXFP8 on Blackwell) and of the ModelScope post's
 // section "精度：FP8 分块量化与净效率收益" (the linear layers' matmuls in FP8).
 //
-// Kernel shape (one CTA per SM, persistent over 128 x 256 output tiles):
+// Kernel shape (one CTA per SM, persistent over 128 x 256 output tiles,
+// 12 warps):
 //   warp 0      TMA producer: A and B K-block tiles (128-byte swizzle) and the
-//               raw scale vectors of each K block, into a 4-stage ring.
+//               raw scale vectors of each K block, into a 3-stage ring.
 //   warp 1      allocates tensor memory; one thread issues tcgen05.mma.
 //   warp 2      scale staging: writes the 128x128-block scale of B into the
 //               ring (FP32 path) or rearranges the UE8M0 scales into the
 //               layout tcgen05.cp copies into tensor memory (block-scaled path).
-//   warps 3-10  epilogue; each owns 32 rows (its TMEM lane quarter) x 128
-//               columns of the tile.
+//   warp 3      spare (keeps the four control warps one per sub-partition).
+//   warps 4-11  epilogue; each owns 32 rows (its TMEM lane quarter) x 128
+//               columns of the tile and its own 8 KB staging buffer, written
+//               in the 128-byte-swizzled layout of a TMA store box.
 // FP32 scales ("promotion" path): each K block's MMAs write a fresh partial
 // product into one of two 256-column TMEM buffers; the epilogue warps load it,
-// multiply by sA * sB and add it into FP32 register accumulators while the
-// tensor core fills the other buffer.  UE8M0 scales: the block-scaled MMA
-// (kind::mxf8f6f4.block_scale) applies the power-of-two scales itself and
-// accumulates the whole K extent in one TMEM buffer; the epilogue drains it
-// into registers once per tile and frees it before converting and storing.
+// multiply by sA * sB and add it into FP32 register accumulators (packed
+// two-wide FMAs) while the tensor core fills the other buffer.  UE8M0 scales:
+// the block-scaled MMA (kind::mxf8f6f4.block_scale) applies the power-of-two
+// scales itself and accumulates the whole K extent in one TMEM buffer; the
+// epilogue drains it into registers once per tile and frees it before
+// converting.  Either way the BF16 tile leaves through shared memory and TMA
+// stores, so the epilogue warps return to the next tile at once.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -43,15 +48,20 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 256;
 constexpr int BK = 128;
-constexpr int STAGES = 4;
-constexpr int kThreads = 352;  // 11 warps
-constexpr int kEpiWarp0 = 3;
+constexpr int STAGES = 3;
+constexpr int kThreads = 384;  // 12 warps: 4 control + 8 epilogue
+constexpr int kEpiWarp0 = 4;
+// Registers are budgeted per SM sub-partition (warp w runs on sub-partition
+// w % 4, 16K registers each): three warps per sub-partition leave 168 per
+// thread, enough for the 128 FP32 accumulators of an epilogue thread plus
+// one 32-column tensor-memory load.
 constexpr int kEpiWarps = 8;
 constexpr int kTmemCols = 512;
 constexpr int kGroupM = 8;  // M blocks per raster group (L2 reuse of B)
 
 constexpr uint32_t kTileABytes = BM * BK;  // 16 KB
 constexpr uint32_t kTileBBytes = BN * BK;  // 32 KB
+constexpr uint32_t kStageBytes = 8192;     // per epilogue warp: 2 boxes of 32 rows x 64 bf16
 // per-stage scale slot
 constexpr uint32_t kSlotRawA = 0;      // 128 FP32 scales (512 B) or 128 UE8M0 bytes
 constexpr uint32_t kSlotRawB = 512;    // 256 FP32 scales (1 KB) or 256 UE8M0 bytes
@@ -61,13 +71,15 @@ constexpr uint32_t kSlotBytes = 3200;  // multiple of 128
 
 constexpr uint32_t kOffA = 0;
 constexpr uint32_t kOffB = kOffA + STAGES * kTileABytes;
-constexpr uint32_t kOffSlot = kOffB + STAGES * kTileBBytes;
+constexpr uint32_t kOffStage = kOffB + STAGES * kTileBBytes;
+constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStageBytes;
 constexpr uint32_t kOffBar = kOffSlot + STAGES * kSlotBytes;
 // barriers: full[S], empty[S], sfready[S], scempty[S], tfull[2], tempty[2], final
 constexpr uint32_t kNumBars = 4 * STAGES + 5;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
 constexpr uint32_t kSmemBytes = kOffMisc + 16;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-B alignment
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
 
 // TMEM columns: FP32 path: partial buffers at 0 and 256.  UE8M0 path: the
 // accumulator at 0..255, then per stage s the A scales at 256 + 16 s (4 cols)
@@ -83,6 +95,7 @@ constexpr int kTimeoutTeardown = 5;
 struct Params {
   CUtensorMap tmA;
   CUtensorMap tmB;
+  CUtensorMap tmD;       // BF16 output, 64 x 32 boxes, 128-byte swizzle
   const void* sA;        // A row-group scales [K/128][lds_a]
   const void* sB;        // B scales (row groups or blocks)
   int64_t sa_stride_k;   // = lds_a
@@ -128,6 +141,40 @@ __device__ __forceinline__ void load_block_scales(const Params& p, int nb, int k
       v0 = __ldg(s + i0);
       v1 = (r0 + 1 < p.nb_blocks) ? __ldg(s + i1) : 127u;
     }
+  }
+}
+
+// Epilogue of one tile for one warp: BF16 conversion of the thread's 128
+// accumulators (row 32*quarter + lane, columns half*128 ...), written into
+// the warp's staging buffer as two 32 x 64 boxes in the 128-byte swizzled
+// layout (16-byte chunk c of row r at chunk position c ^ (r % 8)), then two
+// TMA stores issued by lane 0.  Rows or columns outside D are clipped by TMA.
+__device__ __forceinline__ void store_tile(const Params& p, const float2 (&acc)[64], uint8_t* stage,
+                                           int lane, int m0, int n0) {
+  if (lane == 0) bulk_wait_group_read0();  // the previous tile's stores have left the buffer
+  __syncwarp();
+  const uint32_t sbase = smem_u32(stage);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int q = 32 * j + 4 * c;  // float2 index of columns 64 j + 8 c
+      const uint32_t w0 = pack_bf16x2(acc[q + 0].x, acc[q + 0].y);
+      const uint32_t w1 = pack_bf16x2(acc[q + 1].x, acc[q + 1].y);
+      const uint32_t w2 = pack_bf16x2(acc[q + 2].x, acc[q + 2].y);
+      const uint32_t w3 = pack_bf16x2(acc[q + 3].x, acc[q + 3].y);
+      st_shared_v4(sbase + 4096 * j + 128 * lane + 16 * (c ^ (lane & 7)), w0, w1, w2, w3);
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int x = n0 + 64 * j;
+      if (x < p.N && m0 < p.M) tma_store_2d(&p.tmD, sbase + 4096 * j, x, m0);
+    }
+    bulk_commit_group();
   }
 }
 
@@ -347,22 +394,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         if (lane == 0) mbar_arrive(sfready_bar(s));
       }
     }
-  } else {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     const int ew = warp - kEpiWarp0;   // 0..7
     const int quarter = warp & 3;      // TMEM lane quarter this warp may access
     const int half = ew >> 2;          // column half of the tile
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const int row_in_tile = 32 * quarter + lane;
+    uint8_t* stage = smem + kOffStage + ew * kStageBytes;
     uint32_t it = 0, tcount = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       int mb, nb;
       tile_coords(tile, p.num_m, p.num_n, mb, nb);
-      float acc[128];
+      float2 acc[64];
       if (kFp32) {
 #pragma unroll
-        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -375,31 +423,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           const uint8_t* slot = smem + kOffSlot + s * kSlotBytes;
           const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
           const uint32_t cbase = tmem_base + lane_addr + b * 256 + half * 128;
+          const float2 sa2 = make_float2(sa, sa);
+          float2 f2 = sa2;
           if (!B_ROW) {
             const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[half];
+            f2 = make_float2(f, f);
+          }
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(cbase + 32 * c, r);
-              tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            float r[32];
+            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+            tmem_wait_ld();
+            if (!B_ROW) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) acc[32 * c + i] = fmaf(__uint_as_float(r[i]), f, acc[32 * c + i]);
-            }
-          } else {
-            const float4* sbv = reinterpret_cast<const float4*>(slot + kSlotRawB) + half * 32;
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
+            } else {
+              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(cbase + 32 * c, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 sb = sbv[8 * c + i];
-                acc[32 * c + 4 * i + 0] = fmaf(__uint_as_float(r[4 * i + 0]), sa * sb.x, acc[32 * c + 4 * i + 0]);
-                acc[32 * c + 4 * i + 1] = fmaf(__uint_as_float(r[4 * i + 1]), sa * sb.y, acc[32 * c + 4 * i + 1]);
-                acc[32 * c + 4 * i + 2] = fmaf(__uint_as_float(r[4 * i + 2]), sa * sb.z, acc[32 * c + 4 * i + 2]);
-                acc[32 * c + 4 * i + 3] = fmaf(__uint_as_float(r[4 * i + 3]), sa * sb.w, acc[32 * c + 4 * i + 3]);
-              }
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
+                                             acc[16 * c + i]);
             }
           }
           tc_fence_before();
@@ -415,38 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
         tc_fence_after();
         const uint32_t cbase = tmem_base + lane_addr + half * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(cbase + 32 * c, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) acc[32 * c + i] = __uint_as_float(r[i]);
-        }
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32f(cbase + 32 * c, &acc[16 * c].x);
+        tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(tempty_bar(0));
       }
-      // convert to BF16 (round to nearest even) and store this thread's row
-      const int64_t m = static_cast<int64_t>(mb) * BM + row_in_tile;
-      const int n0 = nb * BN + half * 128;
-      if (m < p.M) {
-        uint16_t* drow = p.D + m * p.ldd + n0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          if (n0 + 8 * c < p.N) {
-            uint4 o;
-            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              uint32_t packed;
-              asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(packed) : "f"(acc[8 * c + 2 * j + 1]), "f"(acc[8 * c + 2 * j]));
-              ow[j] = packed;
-            }
-            *reinterpret_cast<uint4*>(drow + 8 * c) = o;
-          }
-        }
-      }
+      store_tile(p, acc, stage, lane, mb * BM + 32 * quarter, nb * BN + half * 128);
     }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -458,6 +480,370 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   }
 }
 
+// ===================================================== CTA-pair kernel ===
+// Two CTAs of a cluster share every MMA (tcgen05 cta_group::2, M = 256,
+// N = 256): CTA r of the pair holds rows 128 r .. of the 256-row A block, B
+// rows 128 r .. of the 256-row B block, and accumulator rows 128 r .. (all 256
+// columns) in its own TMEM.  Per K block each CTA loads 32 KB instead of the
+// 48 KB of a 128 x 256 tile, so four stages fit beside the epilogue staging
+// and the loads the tensor core waits on are a third smaller.  Roles per CTA
+// are those of the single-CTA kernel; only the even-ranked (leader) CTA's MMA
+// thread issues MMAs.  Barriers:
+//   full[s]    leader; operand bytes of both CTAs (their TMA loads complete
+//              on the leader's barrier), one arrival from the leader's producer
+//   fullsc[s]  local; this CTA's scale vectors
+//   empty[s]   local; arrived by the leader's commit, multicast to both CTAs
+//   sfready[s] local; this CTA's scale staging warp (FP32 promotion path)
+//   sfmma[s]   leader; both staging warps (UE8M0 scale images for tcgen05.cp)
+//   scempty[s] local; this CTA's epilogue warps (scale slot free)
+//   tfull[b]   local; leader's commit, multicast
+//   tempty[b]  leader; the epilogue warps of both CTAs
+// Remote arrivals and waits use the default (CTA-scope) semantics: the
+// barrier phases themselves order the tcgen05 / TMA traffic they guard, and
+// cluster-scope releases or whole-proxy fences cost about a microsecond each.
+namespace pairk {
+constexpr int P_BMC = 128;   // accumulator rows per CTA
+constexpr int P_BN = 256;    // tile columns
+constexpr int P_BNC = 128;   // B rows loaded per CTA
+constexpr int P_STAGES = 4;
+constexpr uint32_t P_kTileA = P_BMC * BK;  // 16 KB
+constexpr uint32_t P_kTileB = P_BNC * BK;  // 16 KB
+constexpr uint32_t P_kOffA = 0;
+constexpr uint32_t P_kOffB = P_kOffA + P_STAGES * P_kTileA;
+constexpr uint32_t P_kOffStage = P_kOffB + P_STAGES * P_kTileB;
+constexpr uint32_t P_kOffSlot = P_kOffStage + kEpiWarps * kStageBytes;
+constexpr uint32_t P_kOffBar = P_kOffSlot + P_STAGES * kSlotBytes;
+// full, fullsc, empty, sfready, sfmma, scempty [S]; tfull[2], tempty[2], final
+constexpr uint32_t P_kNumBars = 6 * P_STAGES + 5;
+constexpr uint32_t P_kOffMisc = P_kOffBar + P_kNumBars * 8;
+constexpr uint32_t P_kSmemBytes = P_kOffMisc + 16;
+constexpr uint32_t P_kSmemAlloc = P_kSmemBytes + 1024;
+static_assert(P_kSmemAlloc <= 232448, "shared memory budget");
+}  // namespace pairk
+
+template <int FMT, bool B_KMAJOR, bool B_ROW>
+__global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_constant__ Params p) {
+  using pairk::P_STAGES;
+  using pairk::P_BMC;
+  using pairk::P_BN;
+  using pairk::P_BNC;
+  using pairk::P_kTileA;
+  using pairk::P_kTileB;
+  using pairk::P_kOffA;
+  using pairk::P_kOffB;
+  using pairk::P_kOffStage;
+  using pairk::P_kOffSlot;
+  using pairk::P_kOffBar;
+  using pairk::P_kOffMisc;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr bool kFp32 = (FMT == kFmtFp32);
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_kOffBar);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto fullsc_bar = [&](int s) { return bar(P_STAGES + s); };
+  auto empty_bar = [&](int s) { return bar(2 * P_STAGES + s); };
+  auto sfready_bar = [&](int s) { return bar(3 * P_STAGES + s); };
+  auto sfmma_bar = [&](int s) { return bar(4 * P_STAGES + s); };
+  auto scempty_bar = [&](int s) { return bar(5 * P_STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar(6 * P_STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar(6 * P_STAGES + 2 + b); };
+  const uint32_t final_bar = bar(6 * P_STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P_kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P_kOffMisc + 4);
+  const WaitGuard guard{abort_flag, p.status, p.limit_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(fullsc_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(sfready_bar(s), 1);
+      mbar_init(sfmma_bar(s), 2);
+      mbar_init(scempty_bar(s), kEpiWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialized, TMEM of both allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int KB = p.num_kb;
+  const int cl = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(nclusters_x());
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&p.tmA);
+      prefetch_tensormap(&p.tmB);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+        int mb, nb;
+        tile_coords(tile, p.num_m, p.num_n, mb, nb);
+        const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
+          if (kFp32 && !mbar_wait(scempty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (P_kTileA + P_kTileB));
+          const uint32_t fb = mapa_shared(full_bar(s), 0);
+          const uint32_t sa = smem_u32(smem + P_kOffA + s * P_kTileA);
+          const uint32_t sb = smem_u32(smem + P_kOffB + s * P_kTileB);
+          tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
+          if (B_KMAJOR)
+            tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, nb * P_BN + P_BNC * static_cast<int>(rank));
+          else
+            tma_load_2d_pair(sb, &p.tmB, fb, nb * P_BN + P_BNC * static_cast<int>(rank), kb * BK);
+          // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
+          uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+          const uint32_t esz = kFp32 ? 4u : 1u;
+          const bool a_sc = row0 < p.sa_stride_k;  // rows past the padded scale rows carry only zeros
+          uint32_t b_sc_bytes = 0;
+          if (B_ROW) {
+            const int64_t left = p.sb_len - static_cast<int64_t>(nb) * P_BN;
+            b_sc_bytes = static_cast<uint32_t>(left < P_BN ? left : P_BN) * esz;
+          }
+          mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz : 0u) + b_sc_bytes);
+          if (a_sc) {
+            const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + (kb * p.sa_stride_k + row0) * esz;
+            bulk_load(smem_u32(slot + kSlotRawA), ga, 128u * esz, fullsc_bar(s));
+          }
+          if (B_ROW) {
+            const uint8_t* gb = static_cast<const uint8_t*>(p.sB) +
+                                (kb * p.sb_stride_k + static_cast<int64_t>(nb) * P_BN) * esz;
+            bulk_load(smem_u32(slot + kSlotRawB), gb, b_sc_bytes, fullsc_bar(s));
+          }
+        }
+      }
+      // teardown: every stage this CTA loaded has been consumed (so its copies
+      // landed) before the CTA exits
+      const uint32_t total = it;
+      for (uint32_t j = (total > P_STAGES ? total - P_STAGES : 0); j < total; ++j) {
+        mbar_wait(empty_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
+        mbar_wait(fullsc_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (leader && lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
+      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
+        if (!kFp32) {
+          if (!mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+        }
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          uint32_t d = tmem_base;
+          if (kFp32) {
+            const uint32_t b = it & 1;
+            if (!mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+            d = tmem_base + b * 256;
+          }
+          if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          if (!kFp32 && !mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + P_kOffA + s * P_kTileA);
+          const uint32_t sb = smem_u32(smem + P_kOffB + s * P_kTileB);
+          const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
+          const uint32_t sf_b = sf_a + 8;
+          if (!kFp32) {
+            const uint32_t tm = smem_u32(smem + P_kOffSlot + s * kSlotBytes + kSlotTm);
+            tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+          }
+#pragma unroll
+          for (int k4 = 0; k4 < BK / 32; ++k4) {
+            const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+            const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                            : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
+            if (kFp32)
+              mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+            else
+              mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(empty_bar(s), 0x3);
+          if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
+        }
+        if (!ok) break;
+        if (!kFp32) tc_commit_pair(tfull_bar(0), 0x3);
+      }
+      tc_commit_pair(final_bar, 0x1);
+      mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------- scale staging
+    uint32_t it = 0;
+    bool ok = true;
+    const uint32_t sfmma_leader_base = mapa_shared(sfmma_bar(0), 0);
+    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
+      if (!B_ROW) {
+        load_block_scales(p, nb, 0, kFp32, cur0, cur1);
+        load_block_scales(p, nb, 32, kFp32, nxt0, nxt1);
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % P_STAGES;
+        const uint32_t ph = (it / P_STAGES) & 1;
+        if (!B_ROW && kb > 0 && (kb & 31) == 0) {
+          cur0 = nxt0;
+          cur1 = nxt1;
+          load_block_scales(p, nb, kb + 32, kFp32, nxt0, nxt1);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), ph, guard, kTimeoutScale))) { ok = false; break; }
+        uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+        uint32_t b0 = 0, b1 = 0;
+        if (!B_ROW) {
+          b0 = __shfl_sync(0xffffffffu, cur0, kb & 31);
+          b1 = __shfl_sync(0xffffffffu, cur1, kb & 31);
+        }
+        if (kFp32) {
+          if (!B_ROW && lane == 0) {
+            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[0] = b0;
+            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[1] = b1;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sfready_bar(s));
+        } else {
+          const uint8_t* ra = slot + kSlotRawA;
+          uint4 wa;
+          wa.x = static_cast<uint32_t>(ra[lane]) * 0x01010101u;
+          wa.y = static_cast<uint32_t>(ra[32 + lane]) * 0x01010101u;
+          wa.z = static_cast<uint32_t>(ra[64 + lane]) * 0x01010101u;
+          wa.w = static_cast<uint32_t>(ra[96 + lane]) * 0x01010101u;
+          *reinterpret_cast<uint4*>(slot + kSlotTm + 16 * lane) = wa;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 wb;
+            if (B_ROW) {
+              const uint8_t* rb = slot + kSlotRawB + 128 * h;
+              wb.x = static_cast<uint32_t>(rb[lane]) * 0x01010101u;
+              wb.y = static_cast<uint32_t>(rb[32 + lane]) * 0x01010101u;
+              wb.z = static_cast<uint32_t>(rb[64 + lane]) * 0x01010101u;
+              wb.w = static_cast<uint32_t>(rb[96 + lane]) * 0x01010101u;
+            } else {
+              const uint32_t v = (h == 0 ? b0 : b1) * 0x01010101u;
+              wb = make_uint4(v, v, v, v);
+            }
+            *reinterpret_cast<uint4*>(slot + kSlotTm + 512 + 512 * h + 16 * lane) = wb;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(sfmma_leader_base + 8 * s);
+        }
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int ew = warp - kEpiWarp0;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
+    const int row_in_tile = 32 * quarter + lane;
+    uint8_t* stage = smem + P_kOffStage + ew * kStageBytes;
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    uint32_t it = 0, tcount = 0;
+    bool ok = true;
+    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      float2 acc[64];
+      if (kFp32) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % P_STAGES;
+          const uint32_t ph = (it / P_STAGES) & 1;
+          const uint32_t b = it & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(b), (it >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(s), ph, guard, kTimeoutEpilogue))) { ok = false; break; }
+          tc_fence_after();
+          const uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+          const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
+          const uint32_t cbase = tmem_base + lane_addr + b * 256 + half * 128;
+          const float2 sa2 = make_float2(sa, sa);
+          float2 f2 = sa2;
+          if (!B_ROW) {
+            const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[half];
+            f2 = make_float2(f, f);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float r[32];
+            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+            tmem_wait_ld();
+            if (!B_ROW) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
+            } else {
+              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
+                                             acc[16 * c + i]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive_cluster(tempty_leader0 + 8 * b);
+            mbar_arrive(scempty_bar(s));
+          }
+        }
+        if (!ok) break;
+      } else {
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(0), tcount & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t cbase = tmem_base + lane_addr + half * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32f(cbase + 32 * c, &acc[16 * c].x);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader0);
+      }
+      const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
+      store_tile(p, acc, stage, lane, m0, nb * P_BN + half * 128);
+    }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // both CTAs done with TMEM, barriers and each other's smem
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------- host --
 __device__ int g_device_status;
 
@@ -465,6 +851,8 @@ struct DeviceInfo {
   int sms = 0;
   int* status = nullptr;
   bool attr_set[8] = {};
+  bool pair_attr_set[8] = {};
+  int pair_clusters[8] = {};
 };
 
 DeviceInfo g_dev[64];
@@ -519,6 +907,46 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
 }
 
 template <int FMT, bool BK_, bool BR_>
+cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cudaStream_t stream) {
+  auto kern = gemm_pair_kernel<FMT, BK_, BR_>;
+  if (!di->pair_attr_set[slot]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pairk::P_kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t occ = {};
+    occ.gridDim = dim3(2 * 148, 1, 1);
+    occ.blockDim = dim3(kThreads, 1, 1);
+    occ.dynamicSmemBytes = pairk::P_kSmemAlloc;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    occ.attrs = attr;
+    occ.numAttrs = 1;
+    int ncl = 0;
+    e = cudaOccupancyMaxActiveClusters(&ncl, kern, &occ);
+    if (e != cudaSuccess) return e;
+    if (ncl <= 0) return cudaErrorInvalidConfiguration;
+    di->pair_clusters[slot] = ncl;
+    di->pair_attr_set[slot] = true;
+  }
+  const int ncl = prm.num_tiles < di->pair_clusters[slot] ? prm.num_tiles : di->pair_clusters[slot];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ncl, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = pairk::P_kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+template <int FMT, bool BK_, bool BR_>
 cudaError_t launch_variant(const Params& prm, int grid, DeviceInfo* di, int slot, cudaStream_t stream) {
   auto kern = gemm_kernel<FMT, BK_, BR_>;
   if (!di->attr_set[slot]) {
@@ -542,13 +970,29 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
 
+  // M <= 128 runs the single-CTA kernel (128 x 256 tiles); larger M runs CTA
+  // pairs (256 x 256 tiles, 128 rows of A and of B per CTA).
+  const bool pair = pr.M > 128;
   Params prm;
   memset(&prm, 0, sizeof(prm));
   if (!encode_2d(&prm.tmA, pr.a.data, pr.K, pr.M, pr.a.ld, BK, BM)) return cudaErrorInvalidValue;
   if (pr.b.k_major) {
-    if (!encode_2d(&prm.tmB, pr.b.data, pr.K, pr.N, pr.b.ld, BK, BN)) return cudaErrorInvalidValue;
+    if (!encode_2d(&prm.tmB, pr.b.data, pr.K, pr.N, pr.b.ld, BK, pair ? pairk::P_BNC : BN))
+      return cudaErrorInvalidValue;
   } else {
     if (!encode_2d(&prm.tmB, pr.b.data, pr.N, pr.K, pr.b.ld, 128, BK)) return cudaErrorInvalidValue;
+  }
+  {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.N), static_cast<cuuint64_t>(pr.M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.ldd) * 2};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(&prm.tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.d, dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   }
   prm.sA = pr.a.scales;
   prm.sB = pr.b.scales;
@@ -562,7 +1006,8 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.M = static_cast<int>(pr.M);
   prm.N = static_cast<int>(pr.N);
   prm.K = static_cast<int>(pr.K);
-  prm.num_m = static_cast<int>((pr.M + BM - 1) / BM);
+  const int64_t tile_m = pair ? 2 * pairk::P_BMC : BM;
+  prm.num_m = static_cast<int>((pr.M + tile_m - 1) / tile_m);
   prm.num_n = static_cast<int>((pr.N + BN - 1) / BN);
   prm.num_tiles = prm.num_m * prm.num_n;
   prm.num_kb = static_cast<int>(pr.K / BK);
@@ -573,6 +1018,16 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   const bool fp32 = pr.fmt == kFmtFp32;
   const bool bk = pr.b.k_major;
   const bool br = pr.b.row_groups;
+  if (pair) {
+    if (fp32) {
+      if (bk && !br) return launch_pair_variant<kFmtFp32, true, false>(prm, di, 0, stream);
+      if (!bk && !br) return launch_pair_variant<kFmtFp32, false, false>(prm, di, 1, stream);
+      return launch_pair_variant<kFmtFp32, true, true>(prm, di, 2, stream);
+    }
+    if (bk && !br) return launch_pair_variant<kFmtUe8m0, true, false>(prm, di, 3, stream);
+    if (!bk && !br) return launch_pair_variant<kFmtUe8m0, false, false>(prm, di, 4, stream);
+    return launch_pair_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
+  }
   if (fp32) {
     if (bk && !br) return launch_variant<kFmtFp32, true, false>(prm, grid, di, 0, stream);
     if (!bk && !br) return launch_variant<kFmtFp32, false, false>(prm, grid, di, 1, stream);

@@ -129,15 +129,19 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t* __rest
   }
   const GroupScale s0 = make_scale<FMT>(m0v);
   const GroupScale s1 = make_scale<FMT>(m1v);
+  float xa[16], xb[16], ya[16], yb[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    xa[i] = bf16_lo(w[i]);
+    xb[i] = bf16_hi(w[i]);
+  }
+  scaled_n<FMT, 16>(xa, s0, ya);
+  scaled_n<FMT, 16>(xb, s1, yb);
   uint32_t a[4], b[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    a[i] = cvt_e4m3x2(scaled<FMT>(bf16_lo(w[4 * i + 0]), s0), scaled<FMT>(bf16_lo(w[4 * i + 1]), s0)) |
-           (cvt_e4m3x2(scaled<FMT>(bf16_lo(w[4 * i + 2]), s0), scaled<FMT>(bf16_lo(w[4 * i + 3]), s0))
-            << 16);
-    b[i] = cvt_e4m3x2(scaled<FMT>(bf16_hi(w[4 * i + 0]), s1), scaled<FMT>(bf16_hi(w[4 * i + 1]), s1)) |
-           (cvt_e4m3x2(scaled<FMT>(bf16_hi(w[4 * i + 2]), s1), scaled<FMT>(bf16_hi(w[4 * i + 3]), s1))
-            << 16);
+    a[i] = cvt_e4m3x2(ya[4 * i + 0], ya[4 * i + 1]) | (cvt_e4m3x2(ya[4 * i + 2], ya[4 * i + 3]) << 16);
+    b[i] = cvt_e4m3x2(yb[4 * i + 0], yb[4 * i + 1]) | (cvt_e4m3x2(yb[4 * i + 2], yb[4 * i + 3]) << 16);
   }
   const int64_t ca = c0 + 2 * p;
   if (ca < K) {

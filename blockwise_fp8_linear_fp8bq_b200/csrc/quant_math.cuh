@@ -34,12 +34,12 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Per-group quantization parameters.  For FP32 scales `mul` is unused and the
-// code takes an IEEE division by `s`; for UE8M0 the code takes an exact
-// multiplication by `mul` = 2^-e.
+// Per-group quantization parameters.  FP32 scales: `s` and, when s is a
+// normal number well above the underflow range, `mul` = RN(1/s) (else 0).
+// UE8M0: `mul` = 2^-e exactly.
 struct GroupScale {
   float s;        // FP32 scale value (FP32 format)
-  float mul;      // 2^-e (UE8M0 format)
+  float mul;      // RN(1/s) (FP32 format) or 2^-e (UE8M0 format)
   uint32_t byte;  // e + 127 (UE8M0 format)
 };
 
@@ -48,7 +48,7 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
   GroupScale g;
   if constexpr (FMT == kFmtFp32) {
     g.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    g.mul = 0.0f;
+    g.mul = (g.s >= 0x1p-125f) ? __frcp_rn(g.s) : 0.0f;
     g.byte = 0;
   } else {
     // From the IEEE fields of amax = 1.f * 2^E:  448 = 1.75 * 2^8, so
@@ -73,22 +73,63 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
   return g;
 }
 
+// fl32(x / s) as far as the E4M3 encoder can tell.  q = RN(x * RN(1/s)) is
+// within 2.5 fp32 ulps of the IEEE quotient RN(x / s) (two roundings of
+// relative size 2^-24 each, plus the quotient's own half ulp).  Every decision
+// boundary of the saturating round-to-nearest-even E4M3 encoder -- a midpoint
+// between neighbouring E4M3 values, including 2^-10 between 0 and the least
+// subnormal -- has at most 5 significant bits, so bits 18..0 of its fp32
+// encoding are zero.  When q is more than 8 encodings away from every such
+// value, q and RN(x / s) lie strictly on the same side of every boundary and
+// encode to the same E4M3 code; otherwise (a fraction ~3e-5 of the values)
+// the IEEE division is taken.  Groups whose scale is too small for a finite
+// reciprocal (mul == 0) always take the IEEE division.
+__device__ __forceinline__ bool near_e4m3_boundary(float q) {
+  return ((__float_as_uint(q) + 8u) & 0x7FFFFu) <= 16u;
+}
+
 template <int FMT>
 __device__ __forceinline__ float scaled(float x, const GroupScale& g) {
-  if constexpr (FMT == kFmtFp32)
-    return __fdiv_rn(x, g.s);
-  else
+  if constexpr (FMT == kFmtFp32) {
+    if (g.mul == 0.0f) return __fdiv_rn(x, g.s);
+    const float q = x * g.mul;
+    return near_e4m3_boundary(q) ? __fdiv_rn(x, g.s) : q;
+  } else {
     return x * g.mul;
+  }
+}
+
+// n values -> their scaled quotients; the IEEE division, when any value
+// needs it, runs in one rarely taken branch rather than per element.
+template <int FMT, int N>
+__device__ __forceinline__ void scaled_n(const float (&x)[N], const GroupScale& g, float (&y)[N]) {
+  if constexpr (FMT == kFmtFp32) {
+    bool slow = (g.mul == 0.0f);
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      y[i] = x[i] * g.mul;
+      slow |= near_e4m3_boundary(y[i]);
+    }
+    if (__builtin_expect(slow, 0)) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) y[i] = scaled<FMT>(x[i], g);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) y[i] = x[i] * g.mul;
+  }
 }
 
 // Eight bf16 (one uint4) -> eight E4M3 codes (one uint2).
 template <int FMT>
 __device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
+  float x[8], y[8];
+  x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
+  x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
+  scaled_n<FMT, 8>(x, g, y);
   uint2 r;
-  r.x = cvt_e4m3x2(scaled<FMT>(bf16_lo(v.x), g), scaled<FMT>(bf16_hi(v.x), g)) |
-        (cvt_e4m3x2(scaled<FMT>(bf16_lo(v.y), g), scaled<FMT>(bf16_hi(v.y), g)) << 16);
-  r.y = cvt_e4m3x2(scaled<FMT>(bf16_lo(v.z), g), scaled<FMT>(bf16_hi(v.z), g)) |
-        (cvt_e4m3x2(scaled<FMT>(bf16_lo(v.w), g), scaled<FMT>(bf16_hi(v.w), g)) << 16);
+  r.x = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
+  r.y = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
   return r;
 }
 

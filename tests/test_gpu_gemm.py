@@ -119,7 +119,8 @@ def test_dgrad_matches_explicit_transpose(fmt):
 
 # ------------------------------------------------------------------- wgrad --
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("shape", [(256, 200, 136), (128, 512, 256), (384, 264, 520)])
+@pytest.mark.parametrize("shape", [(256, 200, 136), (128, 512, 256), (384, 264, 520), (256, 128, 264),
+                                   (512, 96, 128)])
 def test_wgrad_small(fmt, shape):
     M, N, K = shape  # dW[N,K] = dY[M,N]^T X[M,K]
     dy = synth.grads_bf16(M, N, seed=41, device="cuda")
@@ -146,10 +147,12 @@ def integer_bf16(rows, cols, seed):
 
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("kind", ["fwd", "wgrad"])
-def test_exact_integer_accumulation(fmt, kind):
+@pytest.mark.parametrize("M", [256, 128, 600])
+def test_exact_integer_accumulation(fmt, kind, M):
     """FP32 accumulation of exact E4M3 integer products (all sums < 2^24) must be
-    exact: the output equals the int64 product rounded once to BF16."""
-    M, N, K = 256, 384, 1024
+    exact: the output equals the int64 product rounded once to BF16.  M <= 128
+    runs the single-CTA kernel, larger M the CTA-pair kernel."""
+    N, K = 384, 1024
     a = integer_bf16(M, K, 51)
     b = integer_bf16(N, K, 52)
     exact = (a.double() @ b.double().T)
