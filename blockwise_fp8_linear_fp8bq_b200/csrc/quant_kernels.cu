@@ -24,7 +24,7 @@ constexpr int kActRowsPerCta = 64;
 constexpr int kActIters = 4;  // rows per half-warp
 
 template <int FMT>
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M,
+__global__ void __launch_bounds__(256, FMT == kFmtFp32 ? 4 : 5) quant_act_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                         int64_t K, int64_t ldx,
                                                         uint8_t* __restrict__ q,
                                                         void* __restrict__ scales, int64_t lds) {
@@ -45,17 +45,46 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
     else
       v[i] = make_uint4(0, 0, 0, 0);
   }
+  // amax of each (iteration, half) group; lane 2 i + h then computes the
+  // scale of group (i, h) and every lane fetches the scales it needs.
+  float m[kActIters];
+#pragma unroll
+  for (int i = 0; i < kActIters; ++i) {
+    m[i] = amax8(0.0f, v[i]);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+  }
+  GroupScale gs[kActIters];
+  if constexpr (FMT == kFmtFp32) {
+    // an IEEE division and reciprocal per group: computed once per warp
+    float mine = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kActIters; ++i) {
+      const float mi = __shfl_sync(0xffffffffu, m[i], (lane & 1) * 16);
+      if ((lane >> 1) == i) mine = mi;
+    }
+    const GroupScale gmine = make_scale<FMT>(mine);
+#pragma unroll
+    for (int i = 0; i < kActIters; ++i) gs[i] = fetch_scale<FMT>(gmine, 2 * i + half);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kActIters; ++i) gs[i] = make_scale<FMT>(m[i]);
+  }
+
+  uint2 c[kActIters];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < kActIters; ++i) c[i] = quant8_fast<FMT>(v[i], gs[i], slow);
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int i = 0; i < kActIters; ++i) c[i] = quant8_exact<FMT>(v[i], gs[i]);
+  }
 #pragma unroll
   for (int i = 0; i < kActIters; ++i) {
     const int64_t r = row0 + 2 * i + half;
-    float m = amax8(0.0f, v[i]);
-#pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const GroupScale gs = make_scale<FMT>(m);
     if (r < M) {
-      const uint2 c = quant8<FMT>(v[i], gs);
-      *reinterpret_cast<uint2*>(q + r * K + col) = c;
-      if (l16 == 0) store_scale<FMT>(scales, g * lds + r, gs);
+      *reinterpret_cast<uint2*>(q + r * K + col) = c[i];
+      if (l16 == 0) store_scale<FMT>(scales, g * lds + r, gs[i]);
     } else if (r < lds && l16 == 0) {
       store_neutral_scale<FMT>(scales, g * lds + r);
     }
@@ -75,7 +104,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
 constexpr int kTCols = 64;
 
 template <int FMT>
-__global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t* __restrict__ x, int64_t M,
+__global__ void __launch_bounds__(256, FMT == kFmtFp32 ? 4 : 5) quant_act_t_kernel(const uint16_t* __restrict__ x, int64_t M,
                                                           int64_t K, int64_t ldx,
                                                           uint8_t* __restrict__ qt,
                                                           void* __restrict__ scales, int64_t lds) {
@@ -127,22 +156,52 @@ __global__ void __launch_bounds__(256) quant_act_t_kernel(const uint16_t* __rest
     m0v = fmaxf(m0v, __shfl_xor_sync(0xffffffffu, m0v, o));
     m1v = fmaxf(m1v, __shfl_xor_sync(0xffffffffu, m1v, o));
   }
-  const GroupScale s0 = make_scale<FMT>(m0v);
-  const GroupScale s1 = make_scale<FMT>(m1v);
-  float xa[16], xb[16], ya[16], yb[16];
+  // The warp holds 8 groups (4 column pairs x 2 columns); lane 2 a + b
+  // computes the scale of column b of pair a, the others fetch it.
+  GroupScale s0, s1;
+  if constexpr (FMT == kFmtFp32) {
+    const int lane = t & 31;
+    const int a4 = lane >> 3;  // pair within the warp
+    float mine = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    xa[i] = bf16_lo(w[i]);
-    xb[i] = bf16_hi(w[i]);
+    for (int a = 0; a < 4; ++a) {
+      const float t0 = __shfl_sync(0xffffffffu, m0v, 8 * a);
+      const float t1 = __shfl_sync(0xffffffffu, m1v, 8 * a);
+      if (lane == 2 * a) mine = t0;
+      if (lane == 2 * a + 1) mine = t1;
+    }
+    const GroupScale gmine = make_scale<FMT>(mine);
+    s0 = fetch_scale<FMT>(gmine, 2 * a4);
+    s1 = fetch_scale<FMT>(gmine, 2 * a4 + 1);
+  } else {
+    s0 = make_scale<FMT>(m0v);
+    s1 = make_scale<FMT>(m1v);
   }
-  scaled_n<FMT, 16>(xa, s0, ya);
-  scaled_n<FMT, 16>(xb, s1, yb);
-  uint32_t a[4], b[4];
+  uint4 wa[2], wb[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    a[i] = cvt_e4m3x2(ya[4 * i + 0], ya[4 * i + 1]) | (cvt_e4m3x2(ya[4 * i + 2], ya[4 * i + 3]) << 16);
-    b[i] = cvt_e4m3x2(yb[4 * i + 0], yb[4 * i + 1]) | (cvt_e4m3x2(yb[4 * i + 2], yb[4 * i + 3]) << 16);
+  for (int h = 0; h < 2; ++h) {
+    // columns 2p (low halves) and 2p+1 (high halves) of tokens 8h .. 8h+7
+    wa[h] = make_uint4((w[8 * h + 0] & 0xFFFFu) | (w[8 * h + 1] << 16), (w[8 * h + 2] & 0xFFFFu) | (w[8 * h + 3] << 16),
+                       (w[8 * h + 4] & 0xFFFFu) | (w[8 * h + 5] << 16), (w[8 * h + 6] & 0xFFFFu) | (w[8 * h + 7] << 16));
+    wb[h] = make_uint4((w[8 * h + 0] >> 16) | (w[8 * h + 1] & 0xFFFF0000u), (w[8 * h + 2] >> 16) | (w[8 * h + 3] & 0xFFFF0000u),
+                       (w[8 * h + 4] >> 16) | (w[8 * h + 5] & 0xFFFF0000u), (w[8 * h + 6] >> 16) | (w[8 * h + 7] & 0xFFFF0000u));
   }
+  uint2 ca2[2], cb2[2];
+  bool slow = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    ca2[h] = quant8_fast<FMT>(wa[h], s0, slow);
+    cb2[h] = quant8_fast<FMT>(wb[h], s1, slow);
+  }
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      ca2[h] = quant8_exact<FMT>(wa[h], s0);
+      cb2[h] = quant8_exact<FMT>(wb[h], s1);
+    }
+  }
+  uint32_t a[4] = {ca2[0].x, ca2[0].y, ca2[1].x, ca2[1].y};
+  uint32_t b[4] = {cb2[0].x, cb2[0].y, cb2[1].x, cb2[1].y};
   const int64_t ca = c0 + 2 * p;
   if (ca < K) {
     *reinterpret_cast<uint4*>(qt + ca * M + m0 + 16 * j) = make_uint4(a[0], a[1], a[2], a[3]);
@@ -194,10 +253,18 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
 #pragma unroll
   for (int i = 1; i < 8; ++i) m = fmaxf(m, part[i]);
   const GroupScale gs = make_scale<FMT>(m);
+  uint2 c[8];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = quant8_fast<FMT>(v[i], gs, slow);
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c[i] = quant8_exact<FMT>(v[i], gs);
+  }
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t r = nb * 128 + (t >> 4) + 16 * i;
-    if (r < N) *reinterpret_cast<uint2*>(q + r * K + col) = quant8<FMT>(v[i], gs);
+    if (r < N) *reinterpret_cast<uint2*>(q + r * K + col) = c[i];
   }
   if (t == 0) store_scale<FMT>(scales, kb * nnb + nb, gs);
 }

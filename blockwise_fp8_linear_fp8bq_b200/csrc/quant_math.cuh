@@ -34,12 +34,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Per-group quantization parameters.  FP32 scales: `s` and, when s is a
-// normal number well above the underflow range, `mul` = RN(1/s) (else 0).
-// UE8M0: `mul` = 2^-e exactly.
+// Per-group quantization parameters.  FP32 scales: `s`, and the bracketing
+// multipliers mlo / mhi = RN(1/s) * (1 -/+ 2^-20) when s is well above the
+// underflow range (else 0).  UE8M0: `mul` = 2^-e exactly.
 struct GroupScale {
   float s;        // FP32 scale value (FP32 format)
-  float mul;      // RN(1/s) (FP32 format) or 2^-e (UE8M0 format)
+  float mul;      // 2^-e (UE8M0 format); unused for FP32
+  float mlo, mhi; // FP32 format: bracketing multipliers
   uint32_t byte;  // e + 127 (UE8M0 format)
 };
 
@@ -48,7 +49,10 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
   GroupScale g;
   if constexpr (FMT == kFmtFp32) {
     g.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    g.mul = (g.s >= 0x1p-125f) ? __frcp_rn(g.s) : 0.0f;
+    const float r = (g.s >= 0x1p-125f) ? __frcp_rn(g.s) : 0.0f;
+    g.mul = 0.0f;
+    g.mlo = r * (1.0f - 0x1p-20f);
+    g.mhi = r * (1.0f + 0x1p-20f);
     g.byte = 0;
   } else {
     // From the IEEE fields of amax = 1.f * 2^E:  448 = 1.75 * 2^8, so
@@ -68,69 +72,80 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
     }
     g.s = 0.0f;
     g.mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal for e in [-127,127)
+    g.mlo = g.mhi = 0.0f;
     g.byte = static_cast<uint32_t>(e + 127);
   }
   return g;
 }
 
-// fl32(x / s) as far as the E4M3 encoder can tell.  q = RN(x * RN(1/s)) is
-// within 2.5 fp32 ulps of the IEEE quotient RN(x / s) (two roundings of
-// relative size 2^-24 each, plus the quotient's own half ulp).  Every decision
-// boundary of the saturating round-to-nearest-even E4M3 encoder -- a midpoint
-// between neighbouring E4M3 values, including 2^-10 between 0 and the least
-// subnormal -- has at most 5 significant bits, so bits 18..0 of its fp32
-// encoding are zero.  When q is more than 8 encodings away from every such
-// value, q and RN(x / s) lie strictly on the same side of every boundary and
-// encode to the same E4M3 code; otherwise (a fraction ~3e-5 of the values)
-// the IEEE division is taken.  Groups whose scale is too small for a finite
-// reciprocal (mul == 0) always take the IEEE division.
-__device__ __forceinline__ bool near_e4m3_boundary(float q) {
-  return ((__float_as_uint(q) + 8u) & 0x7FFFFu) <= 16u;
-}
-
+// The code of fl32(x / s), found without a division.  With r = RN(1/s)
+// (relative error <= 2^-24), q_lo = RN(x * RN(r (1 - 2^-20))) and
+// q_hi = RN(x * RN(r (1 + 2^-20))) lie within (1 -/+ 2^-20)(1 +/- 3 * 2^-24)
+// of x / s, so |q_lo| < |RN(x / s)| < |q_hi| with the same sign.  The E4M3
+// encoder (round to nearest even, saturating) is monotonic, so when q_lo and
+// q_hi encode to the same code, so does RN(x / s).  Otherwise -- a decision
+// boundary lies in the bracket, for about one value in 2^16 -- the caller
+// recomputes with the IEEE division (quant8_exact), as it does for groups
+// whose scale has no finite reciprocal (mlo == 0).
 template <int FMT>
-__device__ __forceinline__ float scaled(float x, const GroupScale& g) {
-  if constexpr (FMT == kFmtFp32) {
-    if (g.mul == 0.0f) return __fdiv_rn(x, g.s);
-    const float q = x * g.mul;
-    return near_e4m3_boundary(q) ? __fdiv_rn(x, g.s) : q;
-  } else {
-    return x * g.mul;
-  }
-}
-
-// n values -> their scaled quotients; the IEEE division, when any value
-// needs it, runs in one rarely taken branch rather than per element.
-template <int FMT, int N>
-__device__ __forceinline__ void scaled_n(const float (&x)[N], const GroupScale& g, float (&y)[N]) {
-  if constexpr (FMT == kFmtFp32) {
-    bool slow = (g.mul == 0.0f);
-#pragma unroll
-    for (int i = 0; i < N; ++i) {
-      y[i] = x[i] * g.mul;
-      slow |= near_e4m3_boundary(y[i]);
-    }
-    if (__builtin_expect(slow, 0)) {
-#pragma unroll
-      for (int i = 0; i < N; ++i) y[i] = scaled<FMT>(x[i], g);
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < N; ++i) y[i] = x[i] * g.mul;
-  }
-}
-
-// Eight bf16 (one uint4) -> eight E4M3 codes (one uint2).
-template <int FMT>
-__device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
-  float x[8], y[8];
+__device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g, bool& slow) {
+  float x[8];
   x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
   x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
-  scaled_n<FMT, 8>(x, g, y);
+  uint2 r;
+  if constexpr (FMT == kFmtFp32) {
+    uint2 h;
+    r.x = cvt_e4m3x2(x[0] * g.mlo, x[1] * g.mlo) | (cvt_e4m3x2(x[2] * g.mlo, x[3] * g.mlo) << 16);
+    r.y = cvt_e4m3x2(x[4] * g.mlo, x[5] * g.mlo) | (cvt_e4m3x2(x[6] * g.mlo, x[7] * g.mlo) << 16);
+    h.x = cvt_e4m3x2(x[0] * g.mhi, x[1] * g.mhi) | (cvt_e4m3x2(x[2] * g.mhi, x[3] * g.mhi) << 16);
+    h.y = cvt_e4m3x2(x[4] * g.mhi, x[5] * g.mhi) | (cvt_e4m3x2(x[6] * g.mhi, x[7] * g.mhi) << 16);
+    slow |= (r.x != h.x) | (r.y != h.y) | (g.mlo == 0.0f);
+  } else {
+    r.x = cvt_e4m3x2(x[0] * g.mul, x[1] * g.mul) | (cvt_e4m3x2(x[2] * g.mul, x[3] * g.mul) << 16);
+    r.y = cvt_e4m3x2(x[4] * g.mul, x[5] * g.mul) | (cvt_e4m3x2(x[6] * g.mul, x[7] * g.mul) << 16);
+  }
+  return r;
+}
+
+// Eight bf16 -> eight E4M3 codes of fl32(x / s) with the IEEE division for
+// every value near a boundary.  Kept out of line: it runs only on the rare
+// exact path, and inlined copies would raise every kernel's register count.
+template <int FMT>
+static __device__ __noinline__ uint2 quant8_exact_outlined(uint4 v, float s, float mul) {
+  float y[8];
+  const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                      bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = (FMT == kFmtFp32) ? __fdiv_rn(x[i], s) : x[i] * mul;
   uint2 r;
   r.x = cvt_e4m3x2(y[0], y[1]) | (cvt_e4m3x2(y[2], y[3]) << 16);
   r.y = cvt_e4m3x2(y[4], y[5]) | (cvt_e4m3x2(y[6], y[7]) << 16);
   return r;
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 quant8_exact(const uint4& v, const GroupScale& g) {
+  return quant8_exact_outlined<FMT>(v, g.s, g.mul);
+}
+
+// Eight bf16 -> eight E4M3 codes (single-value callers; fused quantize-on-load).
+template <int FMT>
+__device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
+  return quant8_exact<FMT>(v, g);
+}
+
+// Group scale for the group whose amax sits in lane `src` of `amax`, computed
+// once per warp: every lane computes the scale of one group (its own amax) and
+// lanes fetch the result from `src`.
+template <int FMT>
+__device__ __forceinline__ GroupScale fetch_scale(const GroupScale& mine, int src) {
+  GroupScale g;
+  g.s = __shfl_sync(0xffffffffu, mine.s, src);
+  g.mul = __shfl_sync(0xffffffffu, mine.mul, src);
+  g.mlo = __shfl_sync(0xffffffffu, mine.mlo, src);
+  g.mhi = __shfl_sync(0xffffffffu, mine.mhi, src);
+  g.byte = __shfl_sync(0xffffffffu, mine.byte, src);
+  return g;
 }
 
 __device__ __forceinline__ float amax8(float m, const uint4& v) {
