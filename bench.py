@@ -396,6 +396,11 @@ def case_launchers(step, fp):
             fp.row_operand(it["qd"], it["sd"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
         out[f"gemm_wgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+        # fused quantize-on-load: BF16 A quantized inside the GEMM
+        out[f"gemm_fwd_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+        out[f"gemm_dgrad_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.bf16_operand(it["dy"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
     return out
 
 

@@ -79,8 +79,8 @@ int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a,
       const bool transposed = op->s_stride_k == 1 && op->s_stride_r >= nkb;
       if (!plain && !transposed) return FP8BQ_ERR_SHAPE;
     }
-  } else {
-    return FP8BQ_ERR_UNSUPPORTED;  // fused quantize-on-load: not built yet
+  } else if (op->gran != FP8BQ_GRAN_ROW_1x128) {
+    return FP8BQ_ERR_UNSUPPORTED;  // BF16 A is quantized in 1x128 row groups
   }
   out->data = op->data;
   out->ld = op->ld;

@@ -844,6 +844,410 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
   }
 }
 
+// ================================================ fused quantize-on-load ===
+// CTA-pair kernel whose A operand arrives in BF16 [M, K] and is quantized in
+// shared memory, K block by K block, with the arithmetic of the 1x128
+// activation quantizer (same group, same scale, same codes).  Per stage the
+// producer TMA-loads the BF16 A tile (two 64-column boxes, 128-byte swizzle)
+// on a CTA-local barrier and the B tile as in the pair kernel; the eight
+// epilogue warps quantize the tile (two threads per 128-long row), write the
+// E4M3 codes in the MMA's swizzled K-major layout and the row scale (FP32
+// ring entry, or the UE8M0 tensor-memory image), and arrive on the leader's
+// `aready` barrier that the MMA thread waits on.  With FP32 scales the same
+// warps alternate between quantizing K block j and promoting K block j - 1.
+// A and B-block scales of the FP32 path sit in rings of kRing entries indexed
+// by iteration, each with its own barrier, so no writer can run a full ring
+// ahead of its reader.
+namespace fusedk {
+constexpr int F_STAGES = 2;
+constexpr int kRing = 4;
+constexpr uint32_t F_kTileAbf = 128 * 128 * 2;  // two 16 KB boxes of 64 bf16 columns
+constexpr uint32_t F_kTileA = 128 * 128;
+constexpr uint32_t F_kTileB = 128 * 128;
+constexpr uint32_t F_kOffAbf = 0;
+constexpr uint32_t F_kOffA = F_kOffAbf + F_STAGES * F_kTileAbf;
+constexpr uint32_t F_kOffB = F_kOffA + F_STAGES * F_kTileA;
+constexpr uint32_t F_kOffStage = F_kOffB + F_STAGES * F_kTileB;
+constexpr uint32_t F_kOffSlot = F_kOffStage + kEpiWarps * kStageBytes;  // per stage: raw B scales, SF images
+constexpr uint32_t F_kOffRing = F_kOffSlot + F_STAGES * kSlotBytes;     // kRing x (128 A scales + 2 B scales)
+constexpr uint32_t F_kRingBytes = 512 + 16;
+constexpr uint32_t F_kOffBar = F_kOffRing + kRing * F_kRingBytes;
+// full, fullsc, empty, sfmma, aready [S]; aconv, sfready [kRing]; tfull[2], tempty[2], final
+constexpr uint32_t F_kNumBars = 5 * F_STAGES + 2 * kRing + 5;
+constexpr uint32_t F_kOffMisc = (F_kOffBar + F_kNumBars * 8 + 15) / 16 * 16;
+constexpr uint32_t F_kSmemBytes = F_kOffMisc + 16;
+constexpr uint32_t F_kSmemAlloc = F_kSmemBytes + 1024;
+static_assert(F_kSmemAlloc <= 232448, "shared memory budget");
+}  // namespace fusedk
+
+// Quantize one 64-column half of row r of the staged BF16 A tile.  The
+// partner thread (lane ^ 1) holds the other half; the two exchange their amax.
+template <int FMT>
+__device__ __forceinline__ void fused_convert_half(uint32_t abf, uint32_t afp8, int r, int h, float* ring_sa,
+                                                   uint8_t* sf_image) {
+  const uint32_t src = abf + h * 16384 + r * 128;
+  const int sw = r & 7;
+  float m = 0.0f;
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m = amax8(m, ld_shared_v4(src + ((c ^ sw) << 4)));
+  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  const GroupScale g = make_scale<FMT>(m);
+  const uint32_t dst = afp8 + r * 128;
+  bool slow = false;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint2 c0 = quant8_fast<FMT>(ld_shared_v4(src + (((2 * k) ^ sw) << 4)), g, slow);
+    const uint2 c1 = quant8_fast<FMT>(ld_shared_v4(src + (((2 * k + 1) ^ sw) << 4)), g, slow);
+    st_shared_v4(dst + (((4 * h + k) ^ sw) << 4), c0.x, c0.y, c1.x, c1.y);
+  }
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint2 c0 = quant8_exact<FMT>(ld_shared_v4(src + (((2 * k) ^ sw) << 4)), g);
+      const uint2 c1 = quant8_exact<FMT>(ld_shared_v4(src + (((2 * k + 1) ^ sw) << 4)), g);
+      st_shared_v4(dst + (((4 * h + k) ^ sw) << 4), c0.x, c0.y, c1.x, c1.y);
+    }
+  }
+  if (h == 0) {
+    if constexpr (FMT == kFmtFp32)
+      ring_sa[r] = g.s;
+    else
+      *reinterpret_cast<uint32_t*>(sf_image + 16 * (r & 31) + 4 * (r >> 5)) = g.byte * 0x01010101u;
+  }
+}
+
+template <int FMT, bool B_KMAJOR, bool B_ROW>
+__global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __grid_constant__ Params p) {
+  using namespace fusedk;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr bool kFp32 = (FMT == kFmtFp32);
+  constexpr int S = F_STAGES;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + F_kOffBar);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto full_bar = [&](int s) { return bar(s); };
+  auto fullsc_bar = [&](int s) { return bar(S + s); };
+  auto empty_bar = [&](int s) { return bar(2 * S + s); };
+  auto sfmma_bar = [&](int s) { return bar(3 * S + s); };
+  auto aready_bar = [&](int s) { return bar(4 * S + s); };
+  auto aconv_bar = [&](int q) { return bar(5 * S + q); };
+  auto sfready_bar = [&](int q) { return bar(5 * S + kRing + q); };
+  auto tfull_bar = [&](int b) { return bar(5 * S + 2 * kRing + b); };
+  auto tempty_bar = [&](int b) { return bar(5 * S + 2 * kRing + 2 + b); };
+  const uint32_t final_bar = bar(5 * S + 2 * kRing + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + F_kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + F_kOffMisc + 4);
+  const WaitGuard guard{abort_flag, p.status, p.limit_ns};
+  auto ring = [&](int q) { return smem + F_kOffRing + q * F_kRingBytes; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(fullsc_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(sfmma_bar(s), 2);
+      mbar_init(aready_bar(s), 2 * kEpiWarps);
+    }
+    for (int q = 0; q < kRing; ++q) {
+      mbar_init(aconv_bar(q), kEpiWarps);
+      mbar_init(sfready_bar(q), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);
+    }
+    mbar_init(final_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_holder), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int KB = p.num_kb;
+  const int cl = static_cast<int>(cluster_id_x());
+  const int ncl = static_cast<int>(nclusters_x());
+  constexpr int BMC = 128, TBN = 256, BNC = 128;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&p.tmA);
+      prefetch_tensormap(&p.tmB);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+        int mb, nb;
+        tile_coords(tile, p.num_m, p.num_n, mb, nb);
+        const int32_t row0 = mb * (2 * BMC) + BMC * static_cast<int>(rank);
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
+          if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * F_kTileB);
+          const uint32_t fb = mapa_shared(full_bar(s), 0);
+          const uint32_t sb = smem_u32(smem + F_kOffB + s * F_kTileB);
+          if (B_KMAJOR)
+            tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, nb * TBN + BNC * static_cast<int>(rank));
+          else
+            tma_load_2d_pair(sb, &p.tmB, fb, nb * TBN + BNC * static_cast<int>(rank), kb * BK);
+          const uint32_t esz = kFp32 ? 4u : 1u;
+          uint32_t b_sc_bytes = 0;
+          if (B_ROW) {
+            const int64_t left = p.sb_len - static_cast<int64_t>(nb) * TBN;
+            b_sc_bytes = static_cast<uint32_t>(left < TBN ? left : TBN) * esz;
+          }
+          mbar_arrive_expect_tx(fullsc_bar(s), F_kTileAbf + b_sc_bytes);
+          const uint32_t sab = smem_u32(smem + F_kOffAbf + s * F_kTileAbf);
+          tma_load_2d(sab, &p.tmA, fullsc_bar(s), kb * BK, row0);
+          tma_load_2d(sab + F_kTileAbf / 2, &p.tmA, fullsc_bar(s), kb * BK + 64, row0);
+          if (B_ROW) {
+            uint8_t* slot = smem + F_kOffSlot + s * kSlotBytes;
+            const uint8_t* gb = static_cast<const uint8_t*>(p.sB) +
+                                (kb * p.sb_stride_k + static_cast<int64_t>(nb) * TBN) * esz;
+            bulk_load(smem_u32(slot + kSlotRawB), gb, b_sc_bytes, fullsc_bar(s));
+          }
+        }
+      }
+      const uint32_t total = it;
+      for (uint32_t j = (total > S ? total - S : 0); j < total; ++j) {
+        mbar_wait(empty_bar(j % S), (j / S) & 1, guard, kTimeoutTeardown);
+        mbar_wait(fullsc_bar(j % S), (j / S) & 1, guard, kTimeoutTeardown);
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------------- MMA
+    if (leader && lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      const uint32_t idesc = kFp32 ? idesc_f8(2 * BMC, TBN, !B_KMAJOR) : idesc_mxf8(2 * BMC, TBN, !B_KMAJOR);
+      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
+        if (!kFp32) {
+          if (!mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+        }
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          uint32_t d = tmem_base;
+          if (kFp32) {
+            const uint32_t b = it & 1;
+            if (!mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+            d = tmem_base + b * 256;
+          }
+          if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          if (!mbar_wait(aready_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          if (!kFp32 && !mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + F_kOffA + s * F_kTileA);
+          const uint32_t sb = smem_u32(smem + F_kOffB + s * F_kTileB);
+          const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
+          const uint32_t sf_b = sf_a + 8;
+          if (!kFp32) {
+            const uint32_t tm = smem_u32(smem + F_kOffSlot + s * kSlotBytes + kSlotTm);
+            tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+          }
+#pragma unroll
+          for (int k4 = 0; k4 < BK / 32; ++k4) {
+            const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+            const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                            : smem_desc(sb + 4096 * k4, F_kTileB, 1024, kLayoutSw128);
+            if (kFp32)
+              mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+            else
+              mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(empty_bar(s), 0x3);
+          if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
+        }
+        if (!ok) break;
+        if (!kFp32) tc_commit_pair(tfull_bar(0), 0x3);
+      }
+      tc_commit_pair(final_bar, 0x1);
+      mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------- B scale staging (A is converted)
+    uint32_t it = 0;
+    bool ok = true;
+    const uint32_t sfmma_leader_base = mapa_shared(sfmma_bar(0), 0);
+    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
+      if (!B_ROW) {
+        load_block_scales(p, nb, 0, kFp32, cur0, cur1);
+        load_block_scales(p, nb, 32, kFp32, nxt0, nxt1);
+      }
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (it / S) & 1;
+        if (!B_ROW && kb > 0 && (kb & 31) == 0) {
+          cur0 = nxt0;
+          cur1 = nxt1;
+          load_block_scales(p, nb, kb + 32, kFp32, nxt0, nxt1);
+        }
+        if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), ph, guard, kTimeoutScale))) { ok = false; break; }
+        uint8_t* slot = smem + F_kOffSlot + s * kSlotBytes;
+        uint32_t b0 = 0, b1 = 0;
+        if (!B_ROW) {
+          b0 = __shfl_sync(0xffffffffu, cur0, kb & 31);
+          b1 = __shfl_sync(0xffffffffu, cur1, kb & 31);
+        }
+        if (kFp32) {
+          const int q = it % kRing;
+          if (!B_ROW && lane == 0) {
+            reinterpret_cast<uint32_t*>(ring(q) + 512)[0] = b0;
+            reinterpret_cast<uint32_t*>(ring(q) + 512)[1] = b1;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sfready_bar(q));
+        } else {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 wb;
+            if (B_ROW) {
+              const uint8_t* rb = slot + kSlotRawB + 128 * h;
+              wb.x = static_cast<uint32_t>(rb[lane]) * 0x01010101u;
+              wb.y = static_cast<uint32_t>(rb[32 + lane]) * 0x01010101u;
+              wb.z = static_cast<uint32_t>(rb[64 + lane]) * 0x01010101u;
+              wb.w = static_cast<uint32_t>(rb[96 + lane]) * 0x01010101u;
+            } else {
+              const uint32_t v = (h == 0 ? b0 : b1) * 0x01010101u;
+              wb = make_uint4(v, v, v, v);
+            }
+            *reinterpret_cast<uint4*>(slot + kSlotTm + 512 + 512 * h + 16 * lane) = wb;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(sfmma_leader_base + 8 * s);
+        }
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------- A quantization + epilogue warps
+    const int ew = warp - kEpiWarp0;
+    const int quarter = warp & 3;
+    const int half = ew >> 2;
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
+    const int row_in_tile = 32 * quarter + lane;
+    const int e = ew * 32 + lane;  // converter thread: row e / 2, column half e % 2
+    uint8_t* stage = smem + F_kOffStage + ew * kStageBytes;
+    const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
+    const uint32_t aready_leader0 = mapa_shared(aready_bar(0), 0);
+    uint32_t it = 0, tcount = 0;
+    bool ok = true;
+
+    // Quantize the BF16 A tile of iteration `ci` (stage ci % S).
+    auto convert = [&](uint32_t ci) -> bool {
+      const int s = ci % S;
+      if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), (ci / S) & 1, guard, kTimeoutEpilogue))) return false;
+      float* ring_sa = reinterpret_cast<float*>(ring(ci % kRing));
+      uint8_t* sf_image = smem + F_kOffSlot + s * kSlotBytes + kSlotTm;
+      fused_convert_half<FMT>(smem_u32(smem + F_kOffAbf + s * F_kTileAbf), smem_u32(smem + F_kOffA + s * F_kTileA),
+                              e >> 1, e & 1, ring_sa, sf_image);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_cluster(aready_leader0 + 8 * s);
+        if (kFp32) mbar_arrive(aconv_bar(ci % kRing));
+      }
+      return true;
+    };
+
+    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      float2 acc[64];
+      const uint32_t it0 = it;
+      if (kFp32) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int j = 0; j <= KB; ++j) {
+          if (j < KB && !convert(it0 + j)) { ok = false; break; }
+          if (j == 0) continue;
+          const uint32_t pi = it0 + j - 1;  // promote K block j - 1
+          const uint32_t b = pi & 1;
+          const int q = pi % kRing;
+          if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(b), (pi >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(aconv_bar(q), (pi / kRing) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(q), (pi / kRing) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+          tc_fence_after();
+          const float sa = reinterpret_cast<const float*>(ring(q))[row_in_tile];
+          const uint8_t* slot = smem + F_kOffSlot + (pi % S) * kSlotBytes;
+          const uint32_t cbase = tmem_base + lane_addr + b * 256 + half * 128;
+          const float2 sa2 = make_float2(sa, sa);
+          float2 f2 = sa2;
+          if (!B_ROW) {
+            const float f = sa * reinterpret_cast<const float*>(ring(q) + 512)[half];
+            f2 = make_float2(f, f);
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            float r[32];
+            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+            tmem_wait_ld();
+            if (!B_ROW) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
+            } else {
+              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
+                                             acc[16 * c + i]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * b);
+        }
+        if (!ok) break;
+        it = it0 + KB;
+      } else {
+        for (int j = 0; j < KB; ++j)
+          if (!convert(it0 + j)) { ok = false; break; }
+        if (!ok) break;
+        it = it0 + KB;
+        if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(0), tcount & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t cbase = tmem_base + lane_addr + half * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32f(cbase + 32 * c, &acc[16 * c].x);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader0);
+      }
+      const int m0 = mb * (2 * BMC) + BMC * static_cast<int>(rank) + 32 * quarter;
+      store_tile(p, acc, stage, lane, m0, nb * TBN + half * 128);
+    }
+    if (lane == 0) bulk_wait_group0();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------- host --
 __device__ int g_device_status;
 
@@ -853,6 +1257,8 @@ struct DeviceInfo {
   bool attr_set[8] = {};
   bool pair_attr_set[8] = {};
   int pair_clusters[8] = {};
+  bool fused_attr_set[8] = {};
+  int fused_clusters[8] = {};
 };
 
 DeviceInfo g_dev[64];
@@ -947,6 +1353,46 @@ cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cud
 }
 
 template <int FMT, bool BK_, bool BR_>
+cudaError_t launch_fused_variant(const Params& prm, DeviceInfo* di, int slot, cudaStream_t stream) {
+  auto kern = gemm_pair_fused_kernel<FMT, BK_, BR_>;
+  if (!di->fused_attr_set[slot]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, fusedk::F_kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t occ = {};
+    occ.gridDim = dim3(2 * 148, 1, 1);
+    occ.blockDim = dim3(kThreads, 1, 1);
+    occ.dynamicSmemBytes = fusedk::F_kSmemAlloc;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    occ.attrs = attr;
+    occ.numAttrs = 1;
+    int ncl = 0;
+    e = cudaOccupancyMaxActiveClusters(&ncl, kern, &occ);
+    if (e != cudaSuccess) return e;
+    if (ncl <= 0) return cudaErrorInvalidConfiguration;
+    di->fused_clusters[slot] = ncl;
+    di->fused_attr_set[slot] = true;
+  }
+  const int ncl = prm.num_tiles < di->fused_clusters[slot] ? prm.num_tiles : di->fused_clusters[slot];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * ncl, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = fusedk::F_kSmemAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+template <int FMT, bool BK_, bool BR_>
 cudaError_t launch_variant(const Params& prm, int grid, DeviceInfo* di, int slot, cudaStream_t stream) {
   auto kern = gemm_kernel<FMT, BK_, BR_>;
   if (!di->attr_set[slot]) {
@@ -962,7 +1408,7 @@ cudaError_t launch_variant(const Params& prm, int grid, DeviceInfo* di, int slot
 
 cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupported) {
   *unsupported = false;
-  if (pr.a.bf16 || !pr.a.k_major || !pr.a.row_groups || (pr.b.row_groups && !pr.b.k_major)) {
+  if (!pr.a.k_major || !pr.a.row_groups || (pr.b.row_groups && !pr.b.k_major)) {
     *unsupported = true;
     return cudaSuccess;
   }
@@ -970,12 +1416,27 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
 
-  // M <= 128 runs the single-CTA kernel (128 x 256 tiles); larger M runs CTA
-  // pairs (256 x 256 tiles, 128 rows of A and of B per CTA).
-  const bool pair = pr.M > 128;
+  // M <= 128 runs the single-CTA kernel (128 x 256 tiles); larger M, and any
+  // BF16 A (fused quantize-on-load), runs CTA pairs (256 x 256 tiles, 128 rows
+  // of A and of B per CTA).
+  const bool fused = pr.a.bf16;
+  const bool pair = fused || pr.M > 128;
   Params prm;
   memset(&prm, 0, sizeof(prm));
-  if (!encode_2d(&prm.tmA, pr.a.data, pr.K, pr.M, pr.a.ld, BK, BM)) return cudaErrorInvalidValue;
+  if (fused) {
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.K), static_cast<cuuint64_t>(pr.M)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.a.ld) * 2};
+    cuuint32_t box[2] = {64, 128};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = fn(&prm.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pr.a.data), dims, strides,
+                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  } else if (!encode_2d(&prm.tmA, pr.a.data, pr.K, pr.M, pr.a.ld, BK, BM)) {
+    return cudaErrorInvalidValue;
+  }
   if (pr.b.k_major) {
     if (!encode_2d(&prm.tmB, pr.b.data, pr.K, pr.N, pr.b.ld, BK, pair ? pairk::P_BNC : BN))
       return cudaErrorInvalidValue;
@@ -1018,6 +1479,16 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   const bool fp32 = pr.fmt == kFmtFp32;
   const bool bk = pr.b.k_major;
   const bool br = pr.b.row_groups;
+  if (fused) {
+    if (fp32) {
+      if (bk && !br) return launch_fused_variant<kFmtFp32, true, false>(prm, di, 0, stream);
+      if (!bk && !br) return launch_fused_variant<kFmtFp32, false, false>(prm, di, 1, stream);
+      return launch_fused_variant<kFmtFp32, true, true>(prm, di, 2, stream);
+    }
+    if (bk && !br) return launch_fused_variant<kFmtUe8m0, true, false>(prm, di, 3, stream);
+    if (!bk && !br) return launch_fused_variant<kFmtUe8m0, false, false>(prm, di, 4, stream);
+    return launch_fused_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
+  }
   if (pair) {
     if (fp32) {
       if (bk && !br) return launch_pair_variant<kFmtFp32, true, false>(prm, di, 0, stream);
