@@ -429,21 +429,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
             const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[half];
             f2 = make_float2(f, f);
           }
+          if (!B_ROW) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float r[32];
-            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
-            tmem_wait_ld();
-            if (!B_ROW) {
+            for (int c = 0; c < 4; ++c) {
+              float r[32];
+              tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+              tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
-            } else {
-              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
+            }
+          } else {
+            // per-column B scales: 16-column loads keep the staging small
+            // enough for the 128 accumulators to stay in registers
+            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64;
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
-                                             acc[16 * c + i]);
+            for (int c = 0; c < 8; ++c) {
+              float r[16];
+              tmem_ld_32x32b_x16f(cbase + 16 * c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                acc[8 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[8 * c + i]),
+                                            acc[8 * c + i]);
             }
           }
           tc_fence_before();
@@ -792,21 +800,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
             const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[half];
             f2 = make_float2(f, f);
           }
+          if (!B_ROW) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float r[32];
-            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
-            tmem_wait_ld();
-            if (!B_ROW) {
+            for (int c = 0; c < 4; ++c) {
+              float r[32];
+              tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+              tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
-            } else {
-              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
+            }
+          } else {
+            // per-column B scales: 16-column loads keep the staging small
+            // enough for the 128 accumulators to stay in registers
+            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64;
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
-                                             acc[16 * c + i]);
+            for (int c = 0; c < 8; ++c) {
+              float r[16];
+              tmem_ld_32x32b_x16f(cbase + 16 * c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                acc[8 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[8 * c + i]),
+                                            acc[8 * c + i]);
             }
           }
           tc_fence_before();
@@ -1194,21 +1210,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
             const float f = sa * reinterpret_cast<const float*>(ring(q) + 512)[half];
             f2 = make_float2(f, f);
           }
+          if (!B_ROW) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            float r[32];
-            tmem_ld_32x32b_x32f(cbase + 32 * c, r);
-            tmem_wait_ld();
-            if (!B_ROW) {
+            for (int c = 0; c < 4; ++c) {
+              float r[32];
+              tmem_ld_32x32b_x32f(cbase + 32 * c, r);
+              tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 16; ++i)
                 acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
-            } else {
-              const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64 + 16 * c;
+            }
+          } else {
+            // per-column B scales: 16-column loads keep the staging small
+            // enough for the 128 accumulators to stay in registers
+            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64;
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[i]),
-                                             acc[16 * c + i]);
+            for (int c = 0; c < 8; ++c) {
+              float r[16];
+              tmem_ld_32x32b_x16f(cbase + 16 * c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                acc[8 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[8 * c + i]),
+                                            acc[8 * c + i]);
             }
           }
           tc_fence_before();
