@@ -652,13 +652,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (leader && lane == 0) {
+    // The whole warp runs the loop, so descriptors and TMEM addresses stay
+    // warp-uniform; one elected lane issues the tcgen05 instructions.
+    if (leader) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
       for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
         if (!kFp32) {
-          if (!mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
         }
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -667,39 +669,44 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           uint32_t d = tmem_base;
           if (kFp32) {
             const uint32_t b = it & 1;
-            if (!mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
             d = tmem_base + b * 256;
           }
-          if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
-          if (!kFp32 && !mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
+          if (!kFp32 && !__all_sync(0xffffffffu, mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + P_kOffA + s * P_kTileA);
           const uint32_t sb = smem_u32(smem + P_kOffB + s * P_kTileB);
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
-          if (!kFp32) {
-            const uint32_t tm = smem_u32(smem + P_kOffSlot + s * kSlotBytes + kSlotTm);
-            tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
-          }
+          if (elect_one()) {
+            if (!kFp32) {
+              const uint32_t tm = smem_u32(smem + P_kOffSlot + s * kSlotBytes + kSlotTm);
+              tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+            }
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 32; ++k4) {
-            const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
-            const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
-                                            : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
-            if (kFp32)
-              mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
-            else
-              mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < BK / 32; ++k4) {
+              const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+              const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                              : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
+              if (kFp32)
+                mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+              else
+                mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            }
+            tc_commit_pair(empty_bar(s), 0x3);
+            if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
           }
-          tc_commit_pair(empty_bar(s), 0x3);
-          if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
+          __syncwarp();
         }
         if (!ok) break;
-        if (!kFp32) tc_commit_pair(tfull_bar(0), 0x3);
+        if (!kFp32 && elect_one()) tc_commit_pair(tfull_bar(0), 0x3);
+        __syncwarp();
       }
-      tc_commit_pair(final_bar, 0x1);
+      if (elect_one()) tc_commit_pair(final_bar, 0x1);
+      __syncwarp();
       mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
     }
   } else if (warp == 2) {
