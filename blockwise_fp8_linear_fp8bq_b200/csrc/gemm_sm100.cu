@@ -178,6 +178,34 @@ __device__ __forceinline__ void store_tile(const Params& p, const float2 (&acc)[
   }
 }
 
+// Same stores through a single 4 KB box buffer: each 64-column box waits for
+// the previous store to have read the buffer.
+__device__ __forceinline__ void store_tile_4k(const Params& p, const float2 (&acc)[64], uint8_t* stage,
+                                              int lane, int m0, int n0) {
+  const uint32_t sbase = smem_u32(stage);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int q = 32 * j + 4 * c;
+      const uint32_t w0 = pack_bf16x2(acc[q + 0].x, acc[q + 0].y);
+      const uint32_t w1 = pack_bf16x2(acc[q + 1].x, acc[q + 1].y);
+      const uint32_t w2 = pack_bf16x2(acc[q + 2].x, acc[q + 2].y);
+      const uint32_t w3 = pack_bf16x2(acc[q + 3].x, acc[q + 3].y);
+      st_shared_v4(sbase + 128 * lane + 16 * (c ^ (lane & 7)), w0, w1, w2, w3);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int x = n0 + 64 * j;
+      if (x < p.N && m0 < p.M) tma_store_2d(&p.tmD, sbase, x, m0);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <int FMT, bool B_KMAJOR, bool B_ROW>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -499,10 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
 // thread issues MMAs.  Barriers:
 //   full[s]    leader; operand bytes of both CTAs (their TMA loads complete
 //              on the leader's barrier), one arrival from the leader's producer
+//              and, UE8M0 path, one from each CTA's scale staging warp once
+//              its tensor-memory scale image is written
 //   fullsc[s]  local; this CTA's scale vectors
 //   empty[s]   local; arrived by the leader's commit, multicast to both CTAs
 //   sfready[s] local; this CTA's scale staging warp (FP32 promotion path)
-//   sfmma[s]   leader; both staging warps (UE8M0 scale images for tcgen05.cp)
 //   scempty[s] local; this CTA's epilogue warps (scale slot free)
 //   tfull[b]   local; leader's commit, multicast
 //   tempty[b]  leader; the epilogue warps of both CTAs
@@ -513,36 +542,39 @@ namespace pairk {
 constexpr int P_BMC = 128;   // accumulator rows per CTA
 constexpr int P_BN = 256;    // tile columns
 constexpr int P_BNC = 128;   // B rows loaded per CTA
-constexpr int P_STAGES = 4;
 constexpr uint32_t P_kTileA = P_BMC * BK;  // 16 KB
 constexpr uint32_t P_kTileB = P_BNC * BK;  // 16 KB
-constexpr uint32_t P_kOffA = 0;
-constexpr uint32_t P_kOffB = P_kOffA + P_STAGES * P_kTileA;
-constexpr uint32_t P_kOffStage = P_kOffB + P_STAGES * P_kTileB;
-constexpr uint32_t P_kOffSlot = P_kOffStage + kEpiWarps * kStageBytes;
-constexpr uint32_t P_kOffBar = P_kOffSlot + P_STAGES * kSlotBytes;
-// full, fullsc, empty, sfready, sfmma, scempty [S]; tfull[2], tempty[2], final
-constexpr uint32_t P_kNumBars = 6 * P_STAGES + 5;
-constexpr uint32_t P_kOffMisc = P_kOffBar + P_kNumBars * 8;
-constexpr uint32_t P_kSmemBytes = P_kOffMisc + 16;
-constexpr uint32_t P_kSmemAlloc = P_kSmemBytes + 1024;
-static_assert(P_kSmemAlloc <= 232448, "shared memory budget");
+// The FP32-scale path keeps 8 KB of output staging per epilogue warp (its
+// epilogue is the busier side); the UE8M0 path stages one 4 KB box at a time
+// and spends the space on a fifth operand stage.
+template <bool FP32>
+struct Cfg {
+  static constexpr int kStages = FP32 ? 4 : 5;
+  static constexpr uint32_t kStage = FP32 ? 8192u : 4096u;
+  static constexpr uint32_t kOffA = 0;
+  static constexpr uint32_t kOffB = kOffA + kStages * P_kTileA;
+  static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
+  static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
+  static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
+  // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final
+  static constexpr uint32_t kNumBars = 5 * kStages + 5;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmemBytes = kOffMisc + 16;
+  static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(kTmemSf + 16 * kStages <= kTmemCols, "scale-factor columns");
+};
 }  // namespace pairk
 
 template <int FMT, bool B_KMAJOR, bool B_ROW>
 __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_constant__ Params p) {
-  using pairk::P_STAGES;
   using pairk::P_BMC;
   using pairk::P_BN;
   using pairk::P_BNC;
   using pairk::P_kTileA;
   using pairk::P_kTileB;
-  using pairk::P_kOffA;
-  using pairk::P_kOffB;
-  using pairk::P_kOffStage;
-  using pairk::P_kOffSlot;
-  using pairk::P_kOffBar;
-  using pairk::P_kOffMisc;
+  using C = pairk::Cfg<FMT == kFmtFp32>;
+  constexpr int P_STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -552,28 +584,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + P_kOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   auto full_bar = [&](int s) { return bar(s); };
   auto fullsc_bar = [&](int s) { return bar(P_STAGES + s); };
   auto empty_bar = [&](int s) { return bar(2 * P_STAGES + s); };
   auto sfready_bar = [&](int s) { return bar(3 * P_STAGES + s); };
-  auto sfmma_bar = [&](int s) { return bar(4 * P_STAGES + s); };
-  auto scempty_bar = [&](int s) { return bar(5 * P_STAGES + s); };
-  auto tfull_bar = [&](int b) { return bar(6 * P_STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar(6 * P_STAGES + 2 + b); };
-  const uint32_t final_bar = bar(6 * P_STAGES + 4);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + P_kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + P_kOffMisc + 4);
+  auto scempty_bar = [&](int s) { return bar(4 * P_STAGES + s); };
+  auto tfull_bar = [&](int b) { return bar(5 * P_STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar(5 * P_STAGES + 2 + b); };
+  const uint32_t final_bar = bar(5 * P_STAGES + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < P_STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      // UE8M0: the scale-staging warps of both CTAs also arrive on full[s]
+      mbar_init(full_bar(s), kFp32 ? 1 : 3);
       mbar_init(fullsc_bar(s), 1);
       mbar_init(empty_bar(s), 1);
       mbar_init(sfready_bar(s), 1);
-      mbar_init(sfmma_bar(s), 2);
       mbar_init(scempty_bar(s), kEpiWarps);
     }
     for (int b = 0; b < 2; ++b) {
@@ -614,15 +645,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           if (kFp32 && !mbar_wait(scempty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
           if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (P_kTileA + P_kTileB));
           const uint32_t fb = mapa_shared(full_bar(s), 0);
-          const uint32_t sa = smem_u32(smem + P_kOffA + s * P_kTileA);
-          const uint32_t sb = smem_u32(smem + P_kOffB + s * P_kTileB);
+          const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
+          const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
           tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
           if (B_KMAJOR)
             tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, nb * P_BN + P_BNC * static_cast<int>(rank));
           else
             tma_load_2d_pair(sb, &p.tmB, fb, nb * P_BN + P_BNC * static_cast<int>(rank), kb * BK);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
-          uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+          uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           const uint32_t esz = kFp32 ? 4u : 1u;
           const bool a_sc = row0 < p.sa_stride_k;  // rows past the padded scale rows carry only zeros
           uint32_t b_sc_bytes = 0;
@@ -673,15 +704,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
             d = tmem_base + b * 256;
           }
           if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
-          if (!kFp32 && !__all_sync(0xffffffffu, mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + P_kOffA + s * P_kTileA);
-          const uint32_t sb = smem_u32(smem + P_kOffB + s * P_kTileB);
+          const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
+          const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
           if (elect_one()) {
             if (!kFp32) {
-              const uint32_t tm = smem_u32(smem + P_kOffSlot + s * kSlotBytes + kSlotTm);
+              const uint32_t tm = smem_u32(smem + C::kOffSlot + s * kSlotBytes + kSlotTm);
               tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
               tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
               tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
@@ -713,7 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     // ------------------------------------------------------- scale staging
     uint32_t it = 0;
     bool ok = true;
-    const uint32_t sfmma_leader_base = mapa_shared(sfmma_bar(0), 0);
+    const uint32_t full_leader_base = mapa_shared(full_bar(0), 0);
     for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
       int mb, nb;
       tile_coords(tile, p.num_m, p.num_n, mb, nb);
@@ -731,7 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           load_block_scales(p, nb, kb + 32, kFp32, nxt0, nxt1);
         }
         if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), ph, guard, kTimeoutScale))) { ok = false; break; }
-        uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+        uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
         uint32_t b0 = 0, b1 = 0;
         if (!B_ROW) {
           b0 = __shfl_sync(0xffffffffu, cur0, kb & 31);
@@ -769,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           }
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(sfmma_leader_base + 8 * s);
+          if (lane == 0) mbar_arrive_cluster(full_leader_base + 8 * s);
         }
       }
     }
@@ -780,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     const int half = ew >> 2;
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const int row_in_tile = 32 * quarter + lane;
-    uint8_t* stage = smem + P_kOffStage + ew * kStageBytes;
+    uint8_t* stage = smem + C::kOffStage + ew * C::kStage;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
     uint32_t it = 0, tcount = 0;
     bool ok = true;
@@ -798,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(b), (it >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
           if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(s), ph, guard, kTimeoutEpilogue))) { ok = false; break; }
           tc_fence_after();
-          const uint8_t* slot = smem + P_kOffSlot + s * kSlotBytes;
+          const uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
           const uint32_t cbase = tmem_base + lane_addr + b * 256 + half * 128;
           const float2 sa2 = make_float2(sa, sa);
@@ -852,7 +882,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
-      store_tile(p, acc, stage, lane, m0, nb * P_BN + half * 128);
+      if (kFp32)
+        store_tile(p, acc, stage, lane, m0, nb * P_BN + half * 128);
+      else
+        store_tile_4k(p, acc, stage, lane, m0, nb * P_BN + half * 128);
     }
     if (lane == 0) bulk_wait_group0();
     __syncwarp();
@@ -1346,13 +1379,14 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
 template <int FMT, bool BK_, bool BR_>
 cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cudaStream_t stream) {
   auto kern = gemm_pair_kernel<FMT, BK_, BR_>;
+  constexpr uint32_t kSmem = pairk::Cfg<FMT == kFmtFp32>::kSmemAlloc;
   if (!di->pair_attr_set[slot]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pairk::P_kSmemAlloc);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t occ = {};
     occ.gridDim = dim3(2 * 148, 1, 1);
     occ.blockDim = dim3(kThreads, 1, 1);
-    occ.dynamicSmemBytes = pairk::P_kSmemAlloc;
+    occ.dynamicSmemBytes = kSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -1371,7 +1405,7 @@ cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cud
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ncl, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = pairk::P_kSmemAlloc;
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
