@@ -178,13 +178,14 @@ __device__ __forceinline__ void store_tile(const Params& p, const float2 (&acc)[
   }
 }
 
-// Same stores through a single 4 KB box buffer: each 64-column box waits for
-// the previous store to have read the buffer.
-__device__ __forceinline__ void store_tile_4k(const Params& p, const float2 (&acc)[64], uint8_t* stage,
-                                              int lane, int m0, int n0) {
+// Same stores for NBOX 64-column boxes through a single 4 KB box buffer: each
+// box waits for the previous store to have read the buffer.
+template <int NBOX>
+__device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)[32 * NBOX], uint8_t* stage,
+                                            int lane, int m0, int n0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
+  for (int j = 0; j < NBOX; ++j) {
     if (lane == 0) bulk_wait_group_read0();
     __syncwarp();
 #pragma unroll
@@ -305,13 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (lane == 0) {
+    // The whole warp runs the loop, so descriptors and TMEM addresses stay
+    // warp-uniform; one elected lane issues the tcgen05 instructions.
+    {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(BM, BN, !B_KMAJOR) : idesc_mxf8(BM, BN, !B_KMAJOR);
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         if (!kFp32) {
-          if (!mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
         }
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -320,42 +323,47 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
           uint32_t d = tmem_base;
           if (kFp32) {
             const uint32_t b = it & 1;
-            if (!mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
-            if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
             d = tmem_base + b * 256;
           } else {
-            if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
-            if (!mbar_wait(sfready_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + kOffA + s * kTileABytes);
           const uint32_t sb = smem_u32(smem + kOffB + s * kTileBBytes);
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
-          if (!kFp32) {
-            const uint32_t tm = smem_u32(smem + kOffSlot + s * kSlotBytes + kSlotTm);
-            tc_cp_32x128b_warpx4(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
-          }
+          if (elect_one()) {
+            if (!kFp32) {
+              const uint32_t tm = smem_u32(smem + kOffSlot + s * kSlotBytes + kSlotTm);
+              tc_cp_32x128b_warpx4(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+            }
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 32; ++k4) {
-            const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
-            const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
-                                            : smem_desc(sb + 4096 * k4, kTileBBytes / 2, 1024, kLayoutSw128);
-            if (kFp32)
-              mma_f8(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
-            else
-              mma_mxf8(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < BK / 32; ++k4) {
+              const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+              const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                              : smem_desc(sb + 4096 * k4, kTileBBytes / 2, 1024, kLayoutSw128);
+              if (kFp32)
+                mma_f8(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+              else
+                mma_mxf8(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            }
+            tc_commit(empty_bar(s));
+            if (kFp32) tc_commit(tfull_bar(it & 1));
           }
-          tc_commit(empty_bar(s));
-          if (kFp32) tc_commit(tfull_bar(it & 1));
+          __syncwarp();
         }
         if (!ok) break;
-        if (!kFp32) tc_commit(tfull_bar(0));
+        if (!kFp32 && elect_one()) tc_commit(tfull_bar(0));
+        __syncwarp();
       }
-      // teardown: all MMAs this thread issued have completed
-      tc_commit(final_bar);
+      // teardown: all MMAs this warp issued have completed
+      if (elect_one()) tc_commit(final_bar);
+      __syncwarp();
       mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
     }
   } else if (warp == 2) {
@@ -544,13 +552,18 @@ constexpr int P_BN = 256;    // tile columns
 constexpr int P_BNC = 128;   // B rows loaded per CTA
 constexpr uint32_t P_kTileA = P_BMC * BK;  // 16 KB
 constexpr uint32_t P_kTileB = P_BNC * BK;  // 16 KB
-// The FP32-scale path keeps 8 KB of output staging per epilogue warp (its
-// epilogue is the busier side); the UE8M0 path stages one 4 KB box at a time
-// and spends the space on a fifth operand stage.
+// Output staging is one 4 KB box per epilogue warp (two boxes stored one
+// after the other), which leaves room for five operand stages.  Eight
+// epilogue warps of 128 columns each.  (Sixteen warps of 64 columns, capped
+// at 96 registers a thread, ran the FP32 promotion slower: it is bound by
+// the FP32 pipe and tensor-memory reads, not by load latency.)
 template <bool FP32>
 struct Cfg {
-  static constexpr int kStages = FP32 ? 4 : 5;
-  static constexpr uint32_t kStage = FP32 ? 8192u : 4096u;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
+  static constexpr int kCols = 256 / (kEpiWarps / 4);  // accumulator columns per epilogue warp
+  static constexpr int kStages = 5;
+  static constexpr uint32_t kStage = 4096u;  // one 32 x 64 bf16 output box per warp
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * P_kTileA;
   static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
@@ -567,7 +580,8 @@ struct Cfg {
 }  // namespace pairk
 
 template <int FMT, bool B_KMAJOR, bool B_ROW>
-__global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ Params p) {
   using pairk::P_BMC;
   using pairk::P_BN;
   using pairk::P_BNC;
@@ -605,11 +619,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
       mbar_init(fullsc_bar(s), 1);
       mbar_init(empty_bar(s), 1);
       mbar_init(sfready_bar(s), 1);
-      mbar_init(scempty_bar(s), kEpiWarps);
+      mbar_init(scempty_bar(s), C::kEpiWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 2 * kEpiWarps);
+      mbar_init(tempty_bar(b), 2 * C::kEpiWarps);
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
@@ -805,9 +819,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     }
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
+    // Warp w reads TMEM lanes 32 (w % 4) .. and a slice of kCols columns.
+    constexpr int kCols = C::kCols;
+    constexpr int kAcc = kCols / 2;
     const int ew = warp - kEpiWarp0;
     const int quarter = warp & 3;
-    const int half = ew >> 2;
+    const int slice = ew >> 2;
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const int row_in_tile = 32 * quarter + lane;
     uint8_t* stage = smem + C::kOffStage + ew * C::kStage;
@@ -817,10 +834,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
     for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
       int mb, nb;
       tile_coords(tile, p.num_m, p.num_n, mb, nb);
-      float2 acc[64];
+      float2 acc[kAcc];
       if (kFp32) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) acc[i] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < kAcc; ++i) acc[i] = make_float2(0.0f, 0.0f);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
@@ -830,16 +847,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           tc_fence_after();
           const uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
-          const uint32_t cbase = tmem_base + lane_addr + b * 256 + half * 128;
+          const uint32_t cbase = tmem_base + lane_addr + b * 256 + slice * kCols;
           const float2 sa2 = make_float2(sa, sa);
-          float2 f2 = sa2;
           if (!B_ROW) {
-            const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[half];
-            f2 = make_float2(f, f);
-          }
-          if (!B_ROW) {
+            // one 128x128 block of B per 128 columns
+            const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[(slice * kCols) >> 7];
+            const float2 f2 = make_float2(f, f);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kCols / 32; ++c) {
               float r[32];
               tmem_ld_32x32b_x32f(cbase + 32 * c, r);
               tmem_wait_ld();
@@ -850,9 +865,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
           } else {
             // per-column B scales: 16-column loads keep the staging small
             // enough for the 128 accumulators to stay in registers
-            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + half * 64;
+            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + slice * kAcc;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
+            for (int c = 0; c < kCols / 16; ++c) {
               float r[16];
               tmem_ld_32x32b_x16f(cbase + 16 * c, r);
               tmem_wait_ld();
@@ -873,19 +888,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_kernel(const __grid_con
       } else {
         if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(0), tcount & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
         tc_fence_after();
-        const uint32_t cbase = tmem_base + lane_addr + half * 128;
+        const uint32_t cbase = tmem_base + lane_addr + slice * kCols;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32f(cbase + 32 * c, &acc[16 * c].x);
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld_32x32b_x32f(cbase + 32 * c, &acc[16 * c].x);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
-      if (kFp32)
-        store_tile(p, acc, stage, lane, m0, nb * P_BN + half * 128);
-      else
-        store_tile_4k(p, acc, stage, lane, m0, nb * P_BN + half * 128);
+      store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
     }
     if (lane == 0) bulk_wait_group0();
     __syncwarp();
@@ -1083,13 +1095,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
-    if (leader && lane == 0) {
+    // Warp-uniform loop; one elected lane issues (as in the pair kernel).
+    if (leader) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(2 * BMC, TBN, !B_KMAJOR) : idesc_mxf8(2 * BMC, TBN, !B_KMAJOR);
       for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
         if (!kFp32) {
-          if (!mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
         }
         for (int kb = 0; kb < KB; ++kb, ++it) {
@@ -1098,40 +1111,45 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
           uint32_t d = tmem_base;
           if (kFp32) {
             const uint32_t b = it & 1;
-            if (!mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
             d = tmem_base + b * 256;
           }
-          if (!mbar_wait(full_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
-          if (!mbar_wait(aready_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
-          if (!kFp32 && !mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma)) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
+          if (!__all_sync(0xffffffffu, mbar_wait(aready_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
+          if (!kFp32 && !__all_sync(0xffffffffu, mbar_wait(sfmma_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + F_kOffA + s * F_kTileA);
           const uint32_t sb = smem_u32(smem + F_kOffB + s * F_kTileB);
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
-          if (!kFp32) {
-            const uint32_t tm = smem_u32(smem + F_kOffSlot + s * kSlotBytes + kSlotTm);
-            tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
-            tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
-          }
+          if (elect_one()) {
+            if (!kFp32) {
+              const uint32_t tm = smem_u32(smem + F_kOffSlot + s * kSlotBytes + kSlotTm);
+              tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+              tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+            }
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 32; ++k4) {
-            const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
-            const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
-                                            : smem_desc(sb + 4096 * k4, F_kTileB, 1024, kLayoutSw128);
-            if (kFp32)
-              mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
-            else
-              mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            for (int k4 = 0; k4 < BK / 32; ++k4) {
+              const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+              const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                              : smem_desc(sb + 4096 * k4, F_kTileB, 1024, kLayoutSw128);
+              if (kFp32)
+                mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+              else
+                mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+            }
+            tc_commit_pair(empty_bar(s), 0x3);
+            if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
           }
-          tc_commit_pair(empty_bar(s), 0x3);
-          if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
+          __syncwarp();
         }
         if (!ok) break;
-        if (!kFp32) tc_commit_pair(tfull_bar(0), 0x3);
+        if (!kFp32 && elect_one()) tc_commit_pair(tfull_bar(0), 0x3);
+        __syncwarp();
       }
-      tc_commit_pair(final_bar, 0x1);
+      if (elect_one()) tc_commit_pair(final_bar, 0x1);
+      __syncwarp();
       mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
     }
   } else if (warp == 2) {
@@ -1385,7 +1403,7 @@ cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cud
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t occ = {};
     occ.gridDim = dim3(2 * 148, 1, 1);
-    occ.blockDim = dim3(kThreads, 1, 1);
+    occ.blockDim = dim3(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1, 1);
     occ.dynamicSmemBytes = kSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1404,7 +1422,7 @@ cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cud
   const int ncl = prm.num_tiles < di->pair_clusters[slot] ? prm.num_tiles : di->pair_clusters[slot];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ncl, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
