@@ -34,13 +34,12 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// Per-group quantization parameters.  FP32 scales: `s`, and the bracketing
-// multipliers mlo / mhi = RN(1/s) * (1 -/+ 2^-20) when s is well above the
-// underflow range (else 0).  UE8M0: `mul` = 2^-e exactly.
+// Per-group quantization parameters.  FP32 scales: `s` and r = RN(1/s) when
+// s is well inside the normal range (else 0).  UE8M0: `mul` = 2^-e exactly.
 struct GroupScale {
   float s;        // FP32 scale value (FP32 format)
+  float r;        // FP32 format: RN(1/s), or 0 for s < 2^-125
   float mul;      // 2^-e (UE8M0 format); unused for FP32
-  float mlo, mhi; // FP32 format: bracketing multipliers
   uint32_t byte;  // e + 127 (UE8M0 format)
 };
 
@@ -49,10 +48,8 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
   GroupScale g;
   if constexpr (FMT == kFmtFp32) {
     g.s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    const float r = (g.s >= 0x1p-125f) ? __frcp_rn(g.s) : 0.0f;
+    g.r = (g.s >= 0x1p-125f) ? __frcp_rn(g.s) : 0.0f;
     g.mul = 0.0f;
-    g.mlo = r * (1.0f - 0x1p-20f);
-    g.mhi = r * (1.0f + 0x1p-20f);
     g.byte = 0;
   } else {
     // From the IEEE fields of amax = 1.f * 2^E:  448 = 1.75 * 2^8, so
@@ -71,22 +68,25 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
       e = e < -127 ? -127 : (e > 127 ? 127 : e);
     }
     g.s = 0.0f;
+    g.r = 0.0f;
     g.mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal for e in [-127,127)
-    g.mlo = g.mhi = 0.0f;
     g.byte = static_cast<uint32_t>(e + 127);
   }
   return g;
 }
 
-// The code of fl32(x / s), found without a division.  With r = RN(1/s)
-// (relative error <= 2^-24), q_lo = RN(x * RN(r (1 - 2^-20))) and
-// q_hi = RN(x * RN(r (1 + 2^-20))) lie within (1 -/+ 2^-20)(1 +/- 3 * 2^-24)
-// of x / s, so |q_lo| < |RN(x / s)| < |q_hi| with the same sign.  The E4M3
-// encoder (round to nearest even, saturating) is monotonic, so when q_lo and
-// q_hi encode to the same code, so does RN(x / s).  Otherwise -- a decision
-// boundary lies in the bracket, for about one value in 2^16 -- the caller
-// recomputes with the IEEE division (quant8_exact), as it does for groups
-// whose scale has no finite reciprocal (mlo == 0).
+// The code of fl32(x / s), found without a division.  With r = RN(1/s) and
+// q = x / s, y0 = RN(x r) lies within 1.5 ulp of q.  One correction
+// y1 = RN(y0 - r RN(s y0 - x)) is then within 1/2 ulp + 2^-22 ulp of q, i.e.
+// a faithful rounding, for which the residual s y1 - x is exact (fused
+// multiply-add); Markstein's theorem (P. Markstein, IBM J. Res. Dev. 34(1),
+// 1990; M. Cornea, J. Harrison, P. Markstein, ARITH-14, 1999) then gives
+// y2 = RN(y1 - r (s y1 - x)) = RN(q) when r = RN(1/s), barring overflow and
+// underflow.  |q| <= 448 rules out overflow; results small enough to
+// underflow all encode to a signed zero either way.  Residuals are taken as
+// s y - x so that fma(s, +-0, -+0) = +0 and fma(-r, +0, +-0) = +-0 keep the
+// sign of a zero input.  Groups with s < 2^-125 (r = 0) set `slow`; the
+// caller then recomputes with the IEEE division (quant8_exact).
 template <int FMT>
 __device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g, bool& slow) {
   float x[8];
@@ -94,12 +94,24 @@ __device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g
   x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
   uint2 r;
   if constexpr (FMT == kFmtFp32) {
-    uint2 h;
-    r.x = cvt_e4m3x2(x[0] * g.mlo, x[1] * g.mlo) | (cvt_e4m3x2(x[2] * g.mlo, x[3] * g.mlo) << 16);
-    r.y = cvt_e4m3x2(x[4] * g.mlo, x[5] * g.mlo) | (cvt_e4m3x2(x[6] * g.mlo, x[7] * g.mlo) << 16);
-    h.x = cvt_e4m3x2(x[0] * g.mhi, x[1] * g.mhi) | (cvt_e4m3x2(x[2] * g.mhi, x[3] * g.mhi) << 16);
-    h.y = cvt_e4m3x2(x[4] * g.mhi, x[5] * g.mhi) | (cvt_e4m3x2(x[6] * g.mhi, x[7] * g.mhi) << 16);
-    slow |= (r.x != h.x) | (r.y != h.y) | (g.mlo == 0.0f);
+    const float2 r2 = make_float2(g.r, g.r);
+    const float2 nr2 = make_float2(-g.r, -g.r);
+    const float2 s2 = make_float2(g.s, g.s);
+    uint32_t c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 xx = make_float2(x[2 * k], x[2 * k + 1]);
+      const float2 nx = make_float2(-x[2 * k], -x[2 * k + 1]);
+      float2 y = __fmul2_rn(xx, r2);
+      float2 e = __ffma2_rn(s2, y, nx);
+      y = __ffma2_rn(nr2, e, y);
+      e = __ffma2_rn(s2, y, nx);
+      y = __ffma2_rn(nr2, e, y);
+      c[k] = cvt_e4m3x2(y.x, y.y);
+    }
+    r.x = c[0] | (c[1] << 16);
+    r.y = c[2] | (c[3] << 16);
+    slow |= (g.r == 0.0f);
   } else {
     r.x = cvt_e4m3x2(x[0] * g.mul, x[1] * g.mul) | (cvt_e4m3x2(x[2] * g.mul, x[3] * g.mul) << 16);
     r.y = cvt_e4m3x2(x[4] * g.mul, x[5] * g.mul) | (cvt_e4m3x2(x[6] * g.mul, x[7] * g.mul) << 16);
@@ -107,9 +119,9 @@ __device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g
   return r;
 }
 
-// Eight bf16 -> eight E4M3 codes of fl32(x / s) with the IEEE division for
-// every value near a boundary.  Kept out of line: it runs only on the rare
-// exact path, and inlined copies would raise every kernel's register count.
+// Eight bf16 -> eight E4M3 codes of fl32(x / s) with the IEEE division.  Kept
+// out of line: it runs only for groups of tiny scale, and inlined copies would
+// raise every kernel's register count.
 template <int FMT>
 static __device__ __noinline__ uint2 quant8_exact_outlined(uint4 v, float s, float mul) {
   float y[8];
@@ -141,9 +153,8 @@ template <int FMT>
 __device__ __forceinline__ GroupScale fetch_scale(const GroupScale& mine, int src) {
   GroupScale g;
   g.s = __shfl_sync(0xffffffffu, mine.s, src);
+  g.r = __shfl_sync(0xffffffffu, mine.r, src);
   g.mul = __shfl_sync(0xffffffffu, mine.mul, src);
-  g.mlo = __shfl_sync(0xffffffffu, mine.mlo, src);
-  g.mhi = __shfl_sync(0xffffffffu, mine.mhi, src);
   g.byte = __shfl_sync(0xffffffffu, mine.byte, src);
   return g;
 }

@@ -117,3 +117,31 @@ def test_full_size_down_and_grads(fmt):
 def test_full_size_lm_head_weight():
     w = synth.weights_bf16(synth.VOCAB, synth.HIDDEN, seed=3201, device="cuda")
     check_weight(w, fp.SCALE_FP32)
+
+
+def every_finite_bf16() -> torch.Tensor:
+    """All finite bf16 bit patterns (both signs), padded to whole 128-groups."""
+    b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    b = b[(b & 0x7F80) != 0x7F80]  # drop Inf / NaN
+    pad = (-len(b)) % 128
+    b = np.concatenate([b, np.zeros(pad, np.uint16)])
+    return torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_every_bf16_value_against_many_group_maxima(fmt):
+    """Every finite bf16 value, quantized inside groups whose amax takes many
+    different values (so x / s lands on E4M3 decision boundaries and ties
+    exactly, as bf16 ratios often do): codes and scales bit-exact."""
+    vals = every_finite_bf16().to("cuda")
+    n = vals.numel() // 128
+    rows = []
+    for j, amax in enumerate([1.0, 1.5, 3.0, 7.0, 448.0, 0.0625, 1e-3, 65280.0, 1.0078125, 2.0 ** -100]):
+        g = vals.view(n, 128).clone()
+        g = torch.where(g.float().abs() > amax, torch.zeros_like(g), g)
+        g[:, 0] = torch.tensor(amax if j % 2 == 0 else -amax, dtype=torch.bfloat16)
+        rows.append(g)
+    x = torch.cat(rows, 0).reshape(-1, 640)  # 5100 groups -> 1020 rows of 5 groups
+    check_act(x, fmt)
+    check_act_t(x[:896], fmt)
+    check_weight(x, fmt)
