@@ -643,57 +643,55 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      prefetch_tensormap(&p.tmA);
-      prefetch_tensormap(&p.tmB);
-      uint32_t it = 0;
-      bool ok = true;
-      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
-        int mb, nb;
-        tile_coords(tile, p.num_m, p.num_n, mb, nb);
-        const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const int s = it % P_STAGES;
-          const uint32_t ph = (it / P_STAGES) & 1;
-          if (!mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
-          if (kFp32 && !mbar_wait(scempty_bar(s), ph ^ 1, guard, kTimeoutProducer)) { ok = false; break; }
+    // Warp-uniform loop; one elected lane issues the copies.
+    prefetch_tensormap(&p.tmA);
+    prefetch_tensormap(&p.tmB);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+      int mb, nb;
+      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
+      const int32_t brow = nb * P_BN + P_BNC * static_cast<int>(rank);
+      const uint32_t esz = kFp32 ? 4u : 1u;
+      const bool a_sc = row0 < p.sa_stride_k;  // rows past the padded scale rows carry only zeros
+      uint32_t b_sc_bytes = 0;
+      if (B_ROW) {
+        const int64_t left = p.sb_len - static_cast<int64_t>(nb) * P_BN;
+        b_sc_bytes = static_cast<uint32_t>(left < P_BN ? left : P_BN) * esz;
+      }
+      const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + row0 * esz;
+      const uint8_t* gb = static_cast<const uint8_t*>(p.sB) + static_cast<int64_t>(nb) * P_BN * esz;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % P_STAGES;
+        const uint32_t ph = (it / P_STAGES) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer))) { ok = false; break; }
+        if (kFp32 && !__all_sync(0xffffffffu, mbar_wait(scempty_bar(s), ph ^ 1, guard, kTimeoutProducer))) { ok = false; break; }
+        if (elect_one()) {
           if (leader) mbar_arrive_expect_tx(full_bar(s), 2 * (P_kTileA + P_kTileB));
           const uint32_t fb = mapa_shared(full_bar(s), 0);
           const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
           const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
           tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
           if (B_KMAJOR)
-            tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, nb * P_BN + P_BNC * static_cast<int>(rank));
+            tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, brow);
           else
-            tma_load_2d_pair(sb, &p.tmB, fb, nb * P_BN + P_BNC * static_cast<int>(rank), kb * BK);
+            tma_load_2d_pair(sb, &p.tmB, fb, brow, kb * BK);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
-          const uint32_t esz = kFp32 ? 4u : 1u;
-          const bool a_sc = row0 < p.sa_stride_k;  // rows past the padded scale rows carry only zeros
-          uint32_t b_sc_bytes = 0;
-          if (B_ROW) {
-            const int64_t left = p.sb_len - static_cast<int64_t>(nb) * P_BN;
-            b_sc_bytes = static_cast<uint32_t>(left < P_BN ? left : P_BN) * esz;
-          }
           mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz : 0u) + b_sc_bytes);
-          if (a_sc) {
-            const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + (kb * p.sa_stride_k + row0) * esz;
-            bulk_load(smem_u32(slot + kSlotRawA), ga, 128u * esz, fullsc_bar(s));
-          }
-          if (B_ROW) {
-            const uint8_t* gb = static_cast<const uint8_t*>(p.sB) +
-                                (kb * p.sb_stride_k + static_cast<int64_t>(nb) * P_BN) * esz;
-            bulk_load(smem_u32(slot + kSlotRawB), gb, b_sc_bytes, fullsc_bar(s));
-          }
+          if (a_sc) bulk_load(smem_u32(slot + kSlotRawA), ga + kb * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
+          if (B_ROW) bulk_load(smem_u32(slot + kSlotRawB), gb + kb * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
         }
+        __syncwarp();
       }
-      // teardown: every stage this CTA loaded has been consumed (so its copies
-      // landed) before the CTA exits
-      const uint32_t total = it;
-      for (uint32_t j = (total > P_STAGES ? total - P_STAGES : 0); j < total; ++j) {
-        mbar_wait(empty_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
-        mbar_wait(fullsc_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
-      }
+    }
+    // teardown: every stage this CTA loaded has been consumed (so its copies
+    // landed) before the CTA exits
+    const uint32_t total = it;
+    for (uint32_t j = (total > P_STAGES ? total - P_STAGES : 0); j < total; ++j) {
+      mbar_wait(empty_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
+      mbar_wait(fullsc_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
@@ -704,10 +702,6 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
       for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
-        if (!kFp32) {
-          if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
-          tc_fence_after();
-        }
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
@@ -723,13 +717,13 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
-          if (elect_one()) {
-            if (!kFp32) {
-              const uint32_t tm = smem_u32(smem + C::kOffSlot + s * kSlotBytes + kSlotTm);
-              tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
-              tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
-              tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
-            }
+          auto issue_sf = [&]() {
+            const uint32_t tm = smem_u32(smem + C::kOffSlot + s * kSlotBytes + kSlotTm);
+            tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
+            tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
+          };
+          auto issue_mma = [&]() {
 #pragma unroll
             for (int k4 = 0; k4 < BK / 32; ++k4) {
               const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
@@ -742,6 +736,19 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             }
             tc_commit_pair(empty_bar(s), 0x3);
             if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
+          };
+          if (!kFp32 && kb == 0) {
+            // first K block of a tile: the scale factors (own TMEM columns)
+            // are copied while the epilogue still drains the accumulator of
+            // the previous tile; the MMAs wait for it
+            if (elect_one()) issue_sf();
+            __syncwarp();
+            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(0), (tcount & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
+            tc_fence_after();
+            if (elect_one()) issue_mma();
+          } else if (elect_one()) {
+            if (!kFp32) issue_sf();
+            issue_mma();
           }
           __syncwarp();
         }
@@ -1590,6 +1597,24 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   if (bk && !br) return launch_variant<kFmtUe8m0, true, false>(prm, grid, di, 3, stream);
   if (!bk && !br) return launch_variant<kFmtUe8m0, false, false>(prm, grid, di, 4, stream);
   return launch_variant<kFmtUe8m0, true, true>(prm, grid, di, 5, stream);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() { return encode_fn(); }
+
+cudaError_t device_sm_count(int* sms) {
+  DeviceInfo* di = nullptr;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  *sms = di->sms;
+  return cudaSuccess;
+}
+
+cudaError_t device_status_word(int** status) {
+  DeviceInfo* di = nullptr;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  *status = di->status;
+  return cudaSuccess;
 }
 
 cudaError_t read_and_clear_device_status(cudaStream_t stream, int* status) {
