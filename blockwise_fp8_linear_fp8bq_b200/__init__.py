@@ -76,6 +76,8 @@ def lib():
             f = getattr(L, name)
             f.restype = i32
             f.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp]
+        L.fp8bq_quantize_act_dual.restype = i32
+        L.fp8bq_quantize_act_dual.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, i32, vp]
         L.fp8bq_gemm.restype = i32
         L.fp8bq_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
                                  i64, i64, ctypes.c_uint32, vp]
@@ -162,6 +164,21 @@ def quantize_act_t(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
                                     _stream(x))
     _raise(st, "fp8bq_quantize_act_t")
     return q, s
+
+
+def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32):
+    """X [M,K] bf16 -> (q, s, qt, st): the outputs of quantize_act and
+    quantize_act_t from one read of X (M and K multiples of 128)."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = _out(None, (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(None, (K // 128, row_scale_ld(M)), _scale_dtype(fmt), x.device)
+    qt = _out(None, (K, M), torch.float8_e4m3fn, x.device)
+    st = _out(None, (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device)
+    rc = lib().fp8bq_quantize_act_dual(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(),
+                                       qt.data_ptr(), st.data_ptr(), fmt, _stream(x))
+    _raise(rc, "fp8bq_quantize_act_dual")
+    return q, s, qt, st
 
 
 def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):

@@ -104,8 +104,8 @@ int fp8bq_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q
   if (K % 128 != 0) return FP8BQ_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_act(x, M, K, ldx, q, scales, fmt,
-                                             reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, nullptr, nullptr, fmt,
+                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int fp8bq_quantize_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt, void* scales,
@@ -116,7 +116,20 @@ int fp8bq_quantize_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void*
   if (K % 8 != 0) return FP8BQ_ERR_ALIGN;
   if (M == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_act_t(x, M, K, ldx, qt, scales, fmt,
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, nullptr, nullptr, qt, scales, fmt,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                            void* qt, void* scales_t, int fmt, fp8bq_stream_t stream) {
+  int st = check_quant_args(x, M, K, ldx, q, scales, fmt);
+  if (st != FP8BQ_OK) return st;
+  st = check_quant_args(x, M, K, ldx, qt, scales_t, fmt);
+  if (st != FP8BQ_OK) return st;
+  if (K % 128 != 0 || M % 128 != 0) return FP8BQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, qt, scales_t, fmt,
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -1,6 +1,8 @@
 // internal.h -- declarations shared by the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <cstdint>
 
@@ -8,12 +10,19 @@ namespace fp8bq {
 
 inline int64_t round_up128(int64_t r) { return (r + 127) / 128 * 128; }
 
-cudaError_t launch_quant_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
-                             int fmt, cudaStream_t stream);
-cudaError_t launch_quant_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt,
-                               void* scales, int fmt, cudaStream_t stream);
 cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q,
                                 void* scales, int fmt, cudaStream_t stream);
+// TMA-fed activation quantizer: row-group codes (q != nullptr), token-group
+// codes (qt != nullptr), or both from one read of X.
+cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
+                               void* qt, void* s_cols, int fmt, cudaStream_t stream);
+
+// Driver entry point of cuTensorMapEncodeTiled (nullptr if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+// Multiprocessor count of the current device (cached).
+cudaError_t device_sm_count(int* sms);
+// Device address of the kernels' status word on the current device.
+cudaError_t device_status_word(int** status);
 
 // A validated GEMM problem, in the library's internal form.
 struct GemmOperand {

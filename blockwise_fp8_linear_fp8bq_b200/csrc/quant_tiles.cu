@@ -1,0 +1,369 @@
+// quant_tiles.cu -- TMA-fed persistent quantizer for activations and output
+// gradients ("Puro-2B: Poor Lab's Qwen2-1.5B Trained on RTX 5090 within
+// $5090", section "方法": activations quantized in groups of 128).
+//
+// One kernel template, three products of the same BF16 tile X[m0:m0+128,
+// k0:k0+128]:
+//   ROWS  1x128 groups along K: codes q [M, K] and scales [K/128][lds_m]
+//         (the forward / dgrad A operand);
+//   COLS  1x128 groups along the tokens M: codes qT [K, M] and scales
+//         [M/128][lds_k] (the wgrad operands);
+//   both  in one pass, reading X once (the backward pass needs both layouts
+//         of dY, and the forward + wgrad both layouts of X).
+//
+// A persistent CTA per SM: one producer warp streams 128x128 tiles with TMA
+// (two 64-column boxes, 128-byte swizzle) into a six-stage ring; sixteen
+// consumer warps quantize out of shared memory and store codes and scales
+// straight from registers.  Every wait is bounded (status word, as in the
+// GEMM).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "quant_math.cuh"
+
+namespace fp8bq {
+namespace {
+
+constexpr int kQStages = 6;
+constexpr int kQConsumers = 16;                 // consumer warps 0..15; warp 16 produces
+constexpr int kQThreads = 32 * (kQConsumers + 1);
+constexpr uint32_t kQBox = 128 * 128;           // 64 bf16 columns x 128 rows: 16 KB
+constexpr uint32_t kQStage = 2 * kQBox;
+constexpr uint32_t kQOffBar = kQStages * kQStage;
+constexpr uint32_t kQNumBars = 2 * kQStages;  // full[S], empty[S]
+constexpr uint32_t kQOffMisc = kQOffBar + kQNumBars * 8;
+constexpr uint32_t kQSmem = kQOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+static_assert(kQSmem <= 232448, "shared memory budget");
+
+constexpr int kQTimeoutProducer = 11;
+constexpr int kQTimeoutConsumer = 12;
+
+struct QParams {
+  CUtensorMap tmX;  // bf16 [M rows, K cols]; box 64 x 128; 128-byte swizzle
+  int64_t M, K;
+  uint8_t* q;       // ROWS: codes [M, K]
+  void* s_rows;     //       scales [K/128][lds_m]
+  int64_t lds_m;
+  uint8_t* qt;      // COLS: codes [K, M]
+  void* s_cols;     //       scales [M/128][lds_k]
+  int64_t lds_k;
+  int tiles_k, num_tiles;
+  int* status;
+  uint64_t limit_ns;
+};
+
+// Byte offset of 16-byte chunk c (0..15, 8 bf16 each) of tile row r: chunks
+// 0..7 in the first box, 8..15 in the second; 128-byte swizzle within a box.
+__device__ __forceinline__ uint32_t tile_chunk(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * kQBox + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Row groups: warp w, half-warp h, lane l16 own rows 8 w + 2 i + h (i < 4),
+// chunk l16 (8 values); the amax is a 16-lane reduction.
+template <int FMT>
+__device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
+                                          int lane) {
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  uint4 v[4];
+  float m[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * warp + 2 * i + half;
+    v[i] = ld_shared_v4(base + tile_chunk(r, l16));
+    m[i] = amax8(0.0f, v[i]);
+#pragma unroll
+    for (int o = 8; o >= 1; o >>= 1) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+  }
+  GroupScale gs[4];
+  if constexpr (FMT == kFmtFp32) {
+    // one scale per group, computed by lane 2 i + h and fetched by the others
+    float mine = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float mi = __shfl_sync(0xffffffffu, m[i], (lane & 1) * 16);
+      if ((lane >> 1) == i) mine = mi;
+    }
+    const GroupScale gmine = make_scale<FMT>(mine);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) gs[i] = fetch_scale<FMT>(gmine, 2 * i + half);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) gs[i] = make_scale<FMT>(m[i]);
+  }
+  uint2 c[4];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = quant8_fast<FMT>(v[i], gs[i], slow);
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = quant8_exact<FMT>(v[i], gs[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = m0 + 8 * warp + 2 * i + half;
+    if (r < p.M) {
+      *reinterpret_cast<uint2*>(p.q + r * p.K + k0 + 8 * l16) = c[i];
+      if (l16 == 0) store_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r, gs[i]);
+    } else if (r < p.lds_m && l16 == 0) {
+      store_neutral_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r);
+    }
+  }
+}
+
+// Byte i of r moves to byte (i + j) mod 16, for 0 <= j < 8.
+__device__ __forceinline__ uint4 rotate_bytes_up(const uint4& r, int j) {
+  uint32_t x0 = r.x, x1 = r.y, x2 = r.z, x3 = r.w;
+  if (j & 4) {
+    const uint32_t t = x3;
+    x3 = x2;
+    x2 = x1;
+    x1 = x0;
+    x0 = t;
+  }
+  const uint32_t sh = 8u * static_cast<uint32_t>(j & 3);
+  return make_uint4(__funnelshift_l(x3, x0, sh), __funnelshift_l(x0, x1, sh), __funnelshift_l(x1, x2, sh),
+                    __funnelshift_l(x2, x3, sh));
+}
+
+// Token groups: warp w takes box w & 1 and its column pairs 4 (w >> 1) ..
+// + 3; lane (a = lane >> 3, j = lane & 7) owns pair a (two columns, one
+// 32-bit word per token) and tokens 16 j .. 16 j + 15, so a column's 128
+// tokens sit in the eight lanes of its pair and the amax is a shuffle
+// reduction.  Lane j visits its tokens starting at 16 j + j: the eight lanes
+// of a pair then read eight different swizzle phases and the warp's 32 reads
+// hit 32 banks.  The codes come out in that rotated order and are rotated
+// back before each lane stores its 16 consecutive tokens (8 lanes: one
+// 128-byte row segment of the transposed codes).
+template <int FMT>
+__device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
+                                          int lane) {
+  const int box = warp & 1;
+  const int a = lane >> 3;
+  const int j = lane & 7;
+  const int chunk = warp >> 1;  // 16-byte chunk holding the warp's 4 pairs
+  const uint32_t cbase = base + box * kQBox + 4 * a;
+  uint32_t w[16];  // w[i]: token 16 j + ((i + j) & 15)
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int r = 16 * j + ((i + j) & 15);
+    w[i] = ld_shared_u32(cbase + r * 128 + ((chunk ^ (r & 7)) << 4));
+  }
+  float m0v = 0.0f, m1v = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    m0v = fmaxf(m0v, fabsf(bf16_lo(w[i])));
+    m1v = fmaxf(m1v, fabsf(bf16_hi(w[i])));
+  }
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) {
+    m0v = fmaxf(m0v, __shfl_xor_sync(0xffffffffu, m0v, o));
+    m1v = fmaxf(m1v, __shfl_xor_sync(0xffffffffu, m1v, o));
+  }
+  GroupScale s0, s1;
+  if constexpr (FMT == kFmtFp32) {
+    // eight groups per warp: lane 2 a' + b computes column b of pair a'
+    float mine = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float t0 = __shfl_sync(0xffffffffu, m0v, 8 * q);
+      const float t1 = __shfl_sync(0xffffffffu, m1v, 8 * q);
+      if (lane == 2 * q) mine = t0;
+      if (lane == 2 * q + 1) mine = t1;
+    }
+    const GroupScale gmine = make_scale<FMT>(mine);
+    s0 = fetch_scale<FMT>(gmine, 2 * a);
+    s1 = fetch_scale<FMT>(gmine, 2 * a + 1);
+  } else {
+    s0 = make_scale<FMT>(m0v);
+    s1 = make_scale<FMT>(m1v);
+  }
+  uint4 wa[2], wb[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    // first column (low halves) and second column (high halves), 8 tokens
+    wa[h] = make_uint4((w[8 * h + 0] & 0xFFFFu) | (w[8 * h + 1] << 16), (w[8 * h + 2] & 0xFFFFu) | (w[8 * h + 3] << 16),
+                       (w[8 * h + 4] & 0xFFFFu) | (w[8 * h + 5] << 16), (w[8 * h + 6] & 0xFFFFu) | (w[8 * h + 7] << 16));
+    wb[h] = make_uint4((w[8 * h + 0] >> 16) | (w[8 * h + 1] & 0xFFFF0000u), (w[8 * h + 2] >> 16) | (w[8 * h + 3] & 0xFFFF0000u),
+                       (w[8 * h + 4] >> 16) | (w[8 * h + 5] & 0xFFFF0000u), (w[8 * h + 6] >> 16) | (w[8 * h + 7] & 0xFFFF0000u));
+  }
+  uint2 ca[2], cb[2];
+  bool slow = false;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    ca[h] = quant8_fast<FMT>(wa[h], s0, slow);
+    cb[h] = quant8_fast<FMT>(wb[h], s1, slow);
+  }
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      ca[h] = quant8_exact<FMT>(wa[h], s0);
+      cb[h] = quant8_exact<FMT>(wb[h], s1);
+    }
+  }
+  const uint4 va = rotate_bytes_up(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), j);
+  const uint4 vb = rotate_bytes_up(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), j);
+  const int64_t c = k0 + 64 * box + 2 * (4 * chunk + a);
+  const int64_t tok = m0 + 16 * j;
+  const int64_t sidx = (m0 >> 7) * p.lds_k + c;
+  if (c < p.K) {
+    *reinterpret_cast<uint4*>(p.qt + c * p.M + tok) = va;
+    if (j == 0) store_scale<FMT>(p.s_cols, sidx, s0);
+  } else if (c < p.lds_k && j == 0) {
+    store_neutral_scale<FMT>(p.s_cols, sidx);
+  }
+  if (c + 1 < p.K) {
+    *reinterpret_cast<uint4*>(p.qt + (c + 1) * p.M + tok) = vb;
+    if (j == 0) store_scale<FMT>(p.s_cols, sidx + 1, s1);
+  } else if (c + 1 < p.lds_k && j == 0) {
+    store_neutral_scale<FMT>(p.s_cols, sidx + 1);
+  }
+}
+
+template <int FMT, bool ROWS, bool COLS>
+__global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_constant__ QParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kQOffBar);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[kQStages + s]); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQOffMisc);
+  const WaitGuard guard{abort_flag, p.status, p.limit_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kQConsumers);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kQConsumers) {
+    // ------------------------------------------------------------ producer
+    prefetch_tensormap(&p.tmX);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % kQStages;
+      const uint32_t ph = (it / kQStages) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kQTimeoutProducer))) { ok = false; break; }
+      if (elect_one()) {
+        const int32_t m0 = (tile / p.tiles_k) * 128;
+        const int32_t k0 = (tile % p.tiles_k) * 128;
+        // a box wholly past K (ragged K, COLS only) is not loaded: its
+        // columns are never stored and form groups of their own
+        const bool second = k0 + 64 < p.K;
+        const uint32_t dst = smem_u32(smem + s * kQStage);
+        mbar_arrive_expect_tx(full_bar(s), second ? kQStage : kQBox);
+        tma_load_2d(dst, &p.tmX, full_bar(s), k0, m0);
+        if (second) tma_load_2d(dst + kQBox, &p.tmX, full_bar(s), k0 + 64, m0);
+      }
+      __syncwarp();
+    }
+    // teardown: every load issued has landed before the CTA exits
+    const uint32_t total = it;
+    for (uint32_t j = (total > kQStages ? total - kQStages : 0); j < total; ++j)
+      mbar_wait(full_bar(j % kQStages), (j / kQStages) & 1, guard, kQTimeoutProducer);
+  } else {
+    // ------------------------------------------------------------ consumers
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % kQStages;
+      const uint32_t ph = (it / kQStages) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kQTimeoutConsumer))) break;
+      const int64_t m0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
+      const int64_t k0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
+      const uint32_t base = smem_u32(smem + s * kQStage);
+      if (ROWS) tile_rows<FMT>(p, base, m0, k0, warp, lane);
+      if (COLS) tile_cols<FMT>(p, base, m0, k0, warp, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+    }
+  }
+}
+
+// 2-D tensor map over bf16 X [rows, cols] (row pitch in bytes); 64 x 128 boxes,
+// 128-byte swizzle; out-of-range elements read as zero.
+bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64_t ldx) {
+  auto fn = tensor_map_encoder();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldx) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int FMT, bool ROWS, bool COLS>
+cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
+  auto kern = quant_tile_kernel<FMT, ROWS, COLS>;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static bool attr_set[64] = {};
+  if (!attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  int sms = 0;
+  e = device_sm_count(&sms);
+  if (e != cudaSuccess) return e;
+  const int grid = prm.num_tiles < sms ? prm.num_tiles : sms;
+  kern<<<grid, kQThreads, kQSmem, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// X [M, K] -> any of: row-group codes q [M, K] + scales [K/128][round_up(M,128)]
+// (q != nullptr), token-group codes qt [K, M] + scales [M/128][round_up(K,128)]
+// (qt != nullptr; M % 128 == 0).  K % 128 == 0 when q is requested.
+cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
+                               void* qt, void* s_cols, int fmt, cudaStream_t stream) {
+  QParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!encode_x(&prm.tmX, x, M, K, ldx)) return cudaErrorInvalidValue;
+  prm.M = M;
+  prm.K = K;
+  prm.q = static_cast<uint8_t*>(q);
+  prm.s_rows = s_rows;
+  prm.lds_m = round_up128(M);
+  prm.qt = static_cast<uint8_t*>(qt);
+  prm.s_cols = s_cols;
+  prm.lds_k = round_up128(K);
+  prm.tiles_k = static_cast<int>((K + 127) / 128);
+  const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  prm.num_tiles = static_cast<int>(tiles);
+  int* status = nullptr;
+  cudaError_t e = device_status_word(&status);
+  if (e != cudaSuccess) return e;
+  prm.status = status;
+  prm.limit_ns = 2000000000ull;
+  const bool rows = q != nullptr, cols = qt != nullptr;
+  if (fmt == kFmtFp32) {
+    if (rows && cols) return launch_tiles<kFmtFp32, true, true>(prm, stream);
+    if (rows) return launch_tiles<kFmtFp32, true, false>(prm, stream);
+    return launch_tiles<kFmtFp32, false, true>(prm, stream);
+  }
+  if (rows && cols) return launch_tiles<kFmtUe8m0, true, true>(prm, stream);
+  if (rows) return launch_tiles<kFmtUe8m0, true, false>(prm, stream);
+  return launch_tiles<kFmtUe8m0, false, true>(prm, stream);
+}
+
+}  // namespace fp8bq

@@ -119,6 +119,22 @@ int fp8bq_quantize_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void*
                          int fmt, fp8bq_stream_t stream);
 
 /*
+ * Both activation layouts from one read of X: exactly the outputs of
+ * fp8bq_quantize_act (q, scales) and fp8bq_quantize_act_t (qt, scales_t) on
+ * the same x, bit for bit.  Training needs both for each linear layer's input
+ * (forward and weight gradient) and for its output gradient (data gradient
+ * and weight gradient); this call reads the BF16 tensor once instead of twice.
+ * The pages have no such call; it is the same method, fused.
+ *   x         BF16 [M, K], leading dimension ldx.
+ *   q         E4M3 [M, K] (ld K); scales [K/128][fp8bq_row_scale_ld(M)].
+ *   qt        E4M3 [K, M] (ld M); scales_t [M/128][fp8bq_row_scale_ld(K)].
+ * Errors: ERR_SHAPE when K % 128 != 0 or M % 128 != 0; otherwise as
+ * fp8bq_quantize_act.
+ */
+int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                            void* qt, void* scales_t, int fmt, fp8bq_stream_t stream);
+
+/*
  * 128x128 weight-block quantization ("方法": weights in 128x128 blocks).
  *   w       BF16 [N, K], leading dimension ldw (ldw >= K, ldw % 8 == 0).
  *   q       E4M3 [N, K], leading dimension K.

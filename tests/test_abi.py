@@ -80,6 +80,23 @@ def test_quantizer_argument_checks(L, fn):
         assert f(P, 5, 0, 0, P, P, 0, None) == OK
 
 
+def test_dual_quantizer_argument_checks(L):
+    f = L.fp8bq_quantize_act_dual
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    assert f(None, 128, 128, 128, P, P, P, P, 0, None) == INVALID
+    assert f(P, 128, 128, 128, None, P, P, P, 0, None) == INVALID
+    assert f(P, 128, 128, 128, P, P, None, P, 0, None) == INVALID
+    assert f(P, 128, 128, 128, P, P, P, None, 0, None) == INVALID
+    assert f(P, 128, 128, 128, P, P, P, P, 3, None) == INVALID
+    assert f(P, 128, 128, 128, P, P, P + 4, P, 0, None) == ALIGN
+    assert f(P, 128, 128, 128, P, P, P, P + 2, 0, None) == ALIGN
+    assert f(P, 100, 128, 128, P, P, P, P, 0, None) == SHAPE   # tokens % 128
+    assert f(P, 128, 100, 104, P, P, P, P, 0, None) == SHAPE   # columns % 128
+    assert f(P, 0, 128, 128, P, P, P, P, 0, None) == OK        # empty: no launch
+
+
 def _op(L, **kw):
     import blockwise_fp8_linear_fp8bq_b200 as fp
     d = dict(data=P, ld=512, dtype=0, k_major=1, scales=P, gran=0, fmt=0, s_stride_k=256, s_stride_r=1)

@@ -145,3 +145,46 @@ def test_every_bf16_value_against_many_group_maxima(fmt):
     check_act(x, fmt)
     check_act_t(x[:896], fmt)
     check_weight(x, fmt)
+
+
+def check_dual(x, fmt):
+    """The dual quantizer equals act and act_t bit for bit (and the oracle)."""
+    q, s, qt, st = fp.quantize_act_dual(x, fmt)
+    torch.cuda.synchronize()
+    qo, so = oracle.quantize_act(bits(x), fmt)
+    qto, sto = oracle.quantize_act_t(bits(x), fmt)
+    assert np.array_equal(u8(q), qo)
+    assert np.array_equal(scale_bytes(s), so.view(np.uint8).reshape(so.shape[0], -1))
+    assert np.array_equal(u8(qt), qto)
+    assert np.array_equal(scale_bytes(st), sto.view(np.uint8).reshape(sto.shape[0], -1))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("shape", [(128, 256), (256, 384), (384, 1024)])
+def test_quantize_act_dual_small(fmt, shape):
+    x = planted(synth.activations_bf16(*shape, seed=15, device="cuda"))
+    x[:, 5] = 0
+    x[:128, 7] = -2.0 ** -121
+    check_dual(x, fmt)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_quantize_act_dual_full_size(fmt):
+    """dY of gate/up [16384, 12288] (dgrad and wgrad operands) and X [16384, 2048]."""
+    check_dual(synth.GATE_UP.dy(3300, device="cuda"), fmt)
+    check_dual(synth.GATE_UP.x(3300, device="cuda"), fmt)
+
+
+def test_quantize_act_dual_matches_separate_calls():
+    x = synth.DOWN.x(3400, device="cuda")
+    for fmt in FMTS:
+        q, s, qt, st = fp.quantize_act_dual(x, fmt)
+        q1, s1 = fp.quantize_act(x, fmt)
+        qt1, st1 = fp.quantize_act_t(x, fmt)
+        torch.cuda.synchronize()
+        assert torch.equal(u8t(q), u8t(q1)) and torch.equal(s.view(torch.uint8), s1.view(torch.uint8))
+        assert torch.equal(u8t(qt), u8t(qt1)) and torch.equal(st.view(torch.uint8), st1.view(torch.uint8))
+
+
+def u8t(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8)
