@@ -3,13 +3,18 @@
 One step = the full hot path over one batch: the four linears of one
 Qwen3-1.7B-like transformer layer (QKV 2048->4096, O 2048->2048, gate/up
 2048->12288, down 6144->2048) at M = 16384 tokens, each with
-  forward  quantize_act(X), quantize_weight(W), GEMM  Y  = X W^T
-  dgrad    quantize_act(dY),                    GEMM dX = dY W   (W^T read in place)
-  wgrad    quantize_act_t(dY), quantize_act_t(X), GEMM dW = dY^T X
-i.e. 20 quantizer and 12 GEMM launches, 4.948 TFLOP of blockwise-FP8 GEMM.
+  forward  quantize_act_dual(X) (row groups for the forward, token groups for
+           wgrad, one read of X), quantize_weight(W), GEMM  Y = X W^T
+  dgrad    quantize_act_dual(dY) (row groups for dgrad, token groups for
+           wgrad),                                GEMM dX = dY W   (W^T read in place)
+  wgrad                                           GEMM dW = dY^T X
+i.e. 12 quantizer and 12 GEMM launches, 4.948 TFLOP of blockwise-FP8 GEMM.
+With --separate-quant the activation layouts come from quantize_act and
+quantize_act_t in separate launches (20 quantizer launches).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--scale fp32|ue8m0]
     python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+    python bench.py --case all|NAME        # single kernels, L2 flushed
 
 Metric: blockwise-FP8 GEMM TFLOP/s of the whole step (GEMM FLOPs / step time
 including the quantizers), with the GEMM kernel's roofline (TFLOP/s vs the
@@ -126,9 +131,10 @@ class ClockSampler:
 class LayerStep:
     """Device buffers and the launch sequence of one step."""
 
-    def __init__(self, fp, fmt, seed, device, only=None):
+    def __init__(self, fp, fmt, seed, device, only=None, dual=True):
         self.fp = fp
         self.fmt = fmt
+        self.dual = dual
         self.items = []
         sdt = torch.float32 if fmt == fp.SCALE_FP32 else torch.uint8
         e4 = torch.float8_e4m3fn
@@ -161,18 +167,23 @@ class LayerStep:
         for it in self.items:
             lin = it["lin"]
             M, K, N = lin.M, lin.K, lin.N
-            tot += M * K * 3 + (K // 128) * M * sb          # act(X)
             tot += N * K * 3 + (K // 128) * ((N + 127) // 128) * sb  # weight(W)
-            tot += M * N * 3 + (N // 128) * M * sb          # act(dY)
-            tot += M * N * 3 + (M // 128) * N * sb          # act_t(dY)
-            tot += M * K * 3 + (M // 128) * K * sb          # act_t(X)
+            if self.dual:
+                # one bf16 read, both code layouts written
+                tot += M * K * 4 + ((K // 128) * M + (M // 128) * K) * sb  # dual(X)
+                tot += M * N * 4 + ((N // 128) * M + (M // 128) * N) * sb  # dual(dY)
+            else:
+                tot += M * K * 3 + (K // 128) * M * sb          # act(X)
+                tot += M * N * 3 + (N // 128) * M * sb          # act(dY)
+                tot += M * N * 3 + (M // 128) * N * sb          # act_t(dY)
+                tot += M * K * 3 + (M // 128) * K * sb          # act_t(X)
         return tot
 
     def gemm_flops(self):
         return sum(3 * it["lin"].flops for it in self.items)
 
     def launches(self):
-        return 8 * len(self.items)
+        return (6 if self.dual else 8) * len(self.items)
 
     def run(self, ev=None):
         """Issue the step on the current stream.  With `ev` (a list), record a
@@ -191,15 +202,22 @@ class LayerStep:
             ev.append((kind, a, b))
 
         for it in self.items:
-            timed("quant", lambda: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
+            if self.dual:
+                timed("quant", lambda: fp.quantize_act_dual(it["x"], f, it["qx"], it["sx"], it["qxt"], it["sxt"]))
+            else:
+                timed("quant", lambda: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
             timed("quant", lambda: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qx"], it["sx"], f),
                                           fp.block_operand(it["qw"], it["sw"], f), it["y"]))
-            timed("quant", lambda: fp.quantize_act(it["dy"], f, it["qd"], it["sd"]))
+            if self.dual:
+                timed("quant", lambda: fp.quantize_act_dual(it["dy"], f, it["qd"], it["sd"], it["qdt"], it["sdt"]))
+            else:
+                timed("quant", lambda: fp.quantize_act(it["dy"], f, it["qd"], it["sd"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qd"], it["sd"], f),
                                           fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
-            timed("quant", lambda: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
-            timed("quant", lambda: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
+            if not self.dual:
+                timed("quant", lambda: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
+                timed("quant", lambda: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qdt"], it["sdt"], f),
                                           fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
 
@@ -214,7 +232,7 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
-    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev)
+    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
 
@@ -390,6 +408,10 @@ def case_launchers(step, fp):
                                       lambda it=it: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
         out[f"quant_act_t:x:{n}"] = ("quant", M * K * 3 + (M // 128) * K * sb,
                                      lambda it=it: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
+        out[f"quant_dual:x:{n}"] = ("quant", M * K * 4 + ((K // 128) * M + (M // 128) * K) * sb,
+                                    lambda it=it: fp.quantize_act_dual(it["x"], f, it["qx"], it["sx"], it["qxt"], it["sxt"]))
+        out[f"quant_dual:dy:{n}"] = ("quant", M * N * 4 + ((N // 128) * M + (M // 128) * N) * sb,
+                                     lambda it=it: fp.quantize_act_dual(it["dy"], f, it["qd"], it["sd"], it["qdt"], it["sdt"]))
         out[f"gemm_fwd:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.row_operand(it["qx"], it["sx"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))
         out[f"gemm_dgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
@@ -468,8 +490,11 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--scale", choices=["fp32", "ue8m0"], default="fp32")
+    ap.add_argument("--scale", choices=["fp32", "ue8m0"], default="ue8m0",
+                    help="scale format; ue8m0 = the MXFP8 route the pages take on Blackwell")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--separate-quant", action="store_true",
+                    help="quantize each activation layout in its own launch instead of the dual pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="time single kernels instead of the step: 'all' or a name such as gemm_fwd:gate_up")
@@ -523,6 +548,8 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
         "config": {"workload": WORKLOAD, "scale_format": args.scale, "tokens": M_TOKENS,
+                   "activation_quant": "separate act / act_t launches" if args.separate_quant
+                   else "dual (one read of X and of dY, both code layouts)",
                    "parallelism": f"replicas{world}", "l2": "flushed between steps (write of 2x L2)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp8_peak, "traffic": traffic,

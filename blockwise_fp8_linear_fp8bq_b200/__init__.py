@@ -166,15 +166,15 @@ def quantize_act_t(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     return q, s
 
 
-def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32):
+def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None, qt=None, st=None):
     """X [M,K] bf16 -> (q, s, qt, st): the outputs of quantize_act and
     quantize_act_t from one read of X (M and K multiples of 128)."""
     _check_bf16(x, "x")
     M, K = x.shape
-    q = _out(None, (M, K), torch.float8_e4m3fn, x.device)
-    s = _out(None, (K // 128, row_scale_ld(M)), _scale_dtype(fmt), x.device)
-    qt = _out(None, (K, M), torch.float8_e4m3fn, x.device)
-    st = _out(None, (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device)
+    q = _out(q, (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(s, (K // 128, row_scale_ld(M)), _scale_dtype(fmt), x.device)
+    qt = _out(qt, (K, M), torch.float8_e4m3fn, x.device)
+    st = _out(st, (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device)
     rc = lib().fp8bq_quantize_act_dual(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(),
                                        qt.data_ptr(), st.data_ptr(), fmt, _stream(x))
     _raise(rc, "fp8bq_quantize_act_dual")
