@@ -26,6 +26,15 @@ __device__ __forceinline__ float amax2(float m, uint32_t w) {
   return fmaxf(m, fmaxf(fabsf(bf16_lo(w)), fabsf(bf16_hi(w))));
 }
 
+// Per bf16 half: max(|a|, |b|) in magnitude; the sign bits of the result are
+// those of a XOR b and carry no meaning (mask them with 0x7FFF7FFF).  One
+// instruction per two values for the group amax of finite inputs.
+__device__ __forceinline__ uint32_t absmax_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 // Two fp32 -> two E4M3 bytes, round-to-nearest-even with saturation to +-448;
 // `lo` lands in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
@@ -113,8 +122,16 @@ __device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g
     r.y = c[2] | (c[3] << 16);
     slow |= (g.r == 0.0f);
   } else {
-    r.x = cvt_e4m3x2(x[0] * g.mul, x[1] * g.mul) | (cvt_e4m3x2(x[2] * g.mul, x[3] * g.mul) << 16);
-    r.y = cvt_e4m3x2(x[4] * g.mul, x[5] * g.mul) | (cvt_e4m3x2(x[6] * g.mul, x[7] * g.mul) << 16);
+    // x * 2^-e is exact (barring underflow to values that encode to zero)
+    const float2 m2 = make_float2(g.mul, g.mul);
+    uint32_t c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 y = __fmul2_rn(make_float2(x[2 * k], x[2 * k + 1]), m2);
+      c[k] = cvt_e4m3x2(y.x, y.y);
+    }
+    r.x = c[0] | (c[1] << 16);
+    r.y = c[2] | (c[3] << 16);
   }
   return r;
 }

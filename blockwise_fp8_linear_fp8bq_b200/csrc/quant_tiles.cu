@@ -76,9 +76,12 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   for (int i = 0; i < 4; ++i) {
     const int r = 8 * warp + 2 * i + half;
     v[i] = ld_shared_v4(base + tile_chunk(r, l16));
-    m[i] = amax8(0.0f, v[i]);
+    // packed |max| of the 8 values, reduced over the 16 lanes of the row
+    uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w));
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+    for (int o = 8; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    m2 &= 0x7FFF7FFFu;
+    m[i] = fmaxf(bf16_lo(m2), bf16_hi(m2));
   }
   GroupScale gs[4];
   if constexpr (FMT == kFmtFp32) {
@@ -154,17 +157,15 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
     const int r = 16 * j + ((i + j) & 15);
     w[i] = ld_shared_u32(cbase + r * 128 + ((chunk ^ (r & 7)) << 4));
   }
-  float m0v = 0.0f, m1v = 0.0f;
+  // packed |max| over the 16 tokens (both columns at once), then over the
+  // 8 lanes of the pair
+  uint32_t m2 = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    m0v = fmaxf(m0v, fabsf(bf16_lo(w[i])));
-    m1v = fmaxf(m1v, fabsf(bf16_hi(w[i])));
-  }
+  for (int i = 0; i < 16; ++i) m2 = absmax_bf16x2(m2, w[i]);
 #pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) {
-    m0v = fmaxf(m0v, __shfl_xor_sync(0xffffffffu, m0v, o));
-    m1v = fmaxf(m1v, __shfl_xor_sync(0xffffffffu, m1v, o));
-  }
+  for (int o = 4; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  m2 &= 0x7FFF7FFFu;
+  const float m0v = bf16_lo(m2), m1v = bf16_hi(m2);
   GroupScale s0, s1;
   if constexpr (FMT == kFmtFp32) {
     // eight groups per warp: lane 2 a' + b computes column b of pair a'
@@ -187,10 +188,10 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     // first column (low halves) and second column (high halves), 8 tokens
-    wa[h] = make_uint4((w[8 * h + 0] & 0xFFFFu) | (w[8 * h + 1] << 16), (w[8 * h + 2] & 0xFFFFu) | (w[8 * h + 3] << 16),
-                       (w[8 * h + 4] & 0xFFFFu) | (w[8 * h + 5] << 16), (w[8 * h + 6] & 0xFFFFu) | (w[8 * h + 7] << 16));
-    wb[h] = make_uint4((w[8 * h + 0] >> 16) | (w[8 * h + 1] & 0xFFFF0000u), (w[8 * h + 2] >> 16) | (w[8 * h + 3] & 0xFFFF0000u),
-                       (w[8 * h + 4] >> 16) | (w[8 * h + 5] & 0xFFFF0000u), (w[8 * h + 6] >> 16) | (w[8 * h + 7] & 0xFFFF0000u));
+    wa[h] = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x5410), __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x5410),
+                       __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x5410), __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x5410));
+    wb[h] = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x7632), __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x7632),
+                       __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x7632), __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x7632));
   }
   uint2 ca[2], cb[2];
   bool slow = false;
