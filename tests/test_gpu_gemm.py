@@ -211,3 +211,40 @@ def test_mlp_backward_full_size(fmt):
 
 def test_no_pending_device_error():
     fp.check()
+
+
+def compare_sampled_on_device(D: torch.Tensor, A_o, B_o, what, nrows=4, ncols=4, nelem=512, seed=0):
+    """compare_sampled for outputs too large to copy to the host whole: the
+    sampled rows, columns and elements are gathered on the device."""
+    torch.cuda.synchronize()
+    M, N = D.shape
+    rows = sample_indices(M, nrows, seed)
+    cols = sample_indices(N, ncols, seed + 1)
+    rng = np.random.default_rng(seed + 2)
+    er = rng.integers(0, M, nelem)
+    ec = rng.integers(0, N, nelem)
+    dev = D.device
+    got = [to_f64(D[torch.from_numpy(rows).to(dev), :]).ravel(),
+           to_f64(D[:, torch.from_numpy(cols).to(dev)]).ravel(),
+           to_f64(D[torch.from_numpy(er).to(dev), torch.from_numpy(ec).to(dev)]).ravel()]
+    block = np.concatenate([oracle.gemm(A_o, B_o, rows=er[i:i + 256], cols=ec[i:i + 256])[
+        np.arange(len(er[i:i + 256])), np.arange(len(er[i:i + 256]))] for i in range(0, nelem, 256)])
+    ref = [oracle.gemm(A_o, B_o, rows=rows).ravel(), oracle.gemm(A_o, B_o, cols=cols).ravel(), block]
+    return assert_close(np.concatenate(got), np.concatenate(ref), what)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_lm_head_forward_full_size(fmt):
+    """The LM head forward of the 28-layer sweep config: X[16384, 2048] times
+    W[151936, 2048]^T (151936 = 1187 * 128 output columns, 4.98 GB of BF16
+    output), sampled against the oracle."""
+    M, K, N = 16384, synth.HIDDEN, synth.VOCAB
+    x = synth.activations_bf16(M, K, seed=4200, device="cuda")
+    w = synth.weights_bf16(N, K, seed=4201, device="cuda")
+    qx, sx = fp.quantize_act(x, fmt)
+    qw, sw = fp.quantize_weight(w, fmt)
+    del x, w
+    D = fp.gemm(fp.row_operand(qx, sx, fmt), fp.block_operand(qw, sw, fmt))
+    compare_sampled_on_device(D, o_row(qx, sx, fmt), o_block(qw, sw, fmt), "lm_head fwd", seed=4200)
+    del D
+    torch.cuda.empty_cache()
