@@ -38,10 +38,15 @@ __global__ void __launch_bounds__(256) quant_weight_kernel(const uint16_t* __res
     else
       v[i] = make_uint4(0, 0, 0, 0);
   }
+  // packed |max| (two bf16 values per instruction), reduced over the warp
+  uint32_t m2 = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m = amax8(m, v[i]);
+  for (int i = 0; i < 8; ++i)
+    m2 = absmax_bf16x2(absmax_bf16x2(m2, v[i].x), absmax_bf16x2(v[i].y, absmax_bf16x2(v[i].z, v[i].w)));
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int o = 16; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  m2 &= 0x7FFF7FFFu;
+  m = fmaxf(bf16_lo(m2), bf16_hi(m2));
   if ((t & 31) == 0) part[t >> 5] = m;
   __syncthreads();
   m = part[0];

@@ -169,10 +169,17 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, const GroupScale& g) {
 template <int FMT>
 __device__ __forceinline__ GroupScale fetch_scale(const GroupScale& mine, int src) {
   GroupScale g;
-  g.s = __shfl_sync(0xffffffffu, mine.s, src);
-  g.r = __shfl_sync(0xffffffffu, mine.r, src);
-  g.mul = __shfl_sync(0xffffffffu, mine.mul, src);
-  g.byte = __shfl_sync(0xffffffffu, mine.byte, src);
+  if constexpr (FMT == kFmtFp32) {
+    g.s = __shfl_sync(0xffffffffu, mine.s, src);
+    g.r = __shfl_sync(0xffffffffu, mine.r, src);
+    g.mul = 0.0f;
+    g.byte = 0;
+  } else {
+    g.s = 0.0f;
+    g.r = 0.0f;
+    g.mul = __shfl_sync(0xffffffffu, mine.mul, src);
+    g.byte = __shfl_sync(0xffffffffu, mine.byte, src);
+  }
   return g;
 }
 

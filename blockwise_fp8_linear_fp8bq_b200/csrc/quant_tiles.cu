@@ -96,6 +96,7 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
 #pragma unroll
     for (int i = 0; i < 4; ++i) gs[i] = fetch_scale<FMT>(gmine, 2 * i + half);
   } else {
+    // a UE8M0 scale is a few integer operations: cheaper than fetching it
 #pragma unroll
     for (int i = 0; i < 4; ++i) gs[i] = make_scale<FMT>(m[i]);
   }
@@ -107,11 +108,13 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
 #pragma unroll
     for (int i = 0; i < 4; ++i) c[i] = quant8_exact<FMT>(v[i], gs[i]);
   }
+  const int64_t r0 = m0 + 8 * warp + half;
+  uint8_t* qrow = p.q + r0 * p.K + k0 + 8 * l16;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int64_t r = m0 + 8 * warp + 2 * i + half;
+    const int64_t r = r0 + 2 * i;
     if (r < p.M) {
-      *reinterpret_cast<uint2*>(p.q + r * p.K + k0 + 8 * l16) = c[i];
+      *reinterpret_cast<uint2*>(qrow + 2 * i * p.K) = c[i];
       if (l16 == 0) store_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r, gs[i]);
     } else if (r < p.lds_m && l16 == 0) {
       store_neutral_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r);
@@ -166,9 +169,9 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   for (int o = 4; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
   m2 &= 0x7FFF7FFFu;
   const float m0v = bf16_lo(m2), m1v = bf16_hi(m2);
+  // eight groups per warp: lane 2 a' + b computes column b of pair a'
   GroupScale s0, s1;
-  if constexpr (FMT == kFmtFp32) {
-    // eight groups per warp: lane 2 a' + b computes column b of pair a'
+  {
     float mine = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -180,9 +183,6 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
     const GroupScale gmine = make_scale<FMT>(mine);
     s0 = fetch_scale<FMT>(gmine, 2 * a);
     s1 = fetch_scale<FMT>(gmine, 2 * a + 1);
-  } else {
-    s0 = make_scale<FMT>(m0v);
-    s1 = make_scale<FMT>(m1v);
   }
   uint4 wa[2], wb[2];
 #pragma unroll
