@@ -34,6 +34,9 @@
  *     scales[cb * round_up(R,128) + r]; pad entries r >= R hold the neutral
  *     scale (1.0f, or byte 127).
  *   - 128x128 blocks: scales[cb * ceil(R/128) + rb].
+ *   - 1x32 row groups (the other reading of "MXFP8 on Blackwell": the OCP
+ *     Microscaling format's 32-element blocks with E8M0 scales): as 1x128
+ *     row groups with 32 in place of 128, scales[cb32 * round_up(R,128) + r].
  *
  * Parity status: every function here is pinned by tests in tests/ (codec
  * against torch's float8_e4m3fn conversion and the closed-form grid,
@@ -55,6 +58,7 @@
 #define OR_SCALE_UE8M0 1
 #define OR_GRAN_ROW 0
 #define OR_GRAN_BLOCK 1
+#define OR_GRAN_ROW32 2
 #define OR_GROUP 128
 
 /* ---------------------------------------------------------------- codec -- */
@@ -172,24 +176,24 @@ static void fill_row_pad(void* scales, int fmt, int64_t R, int64_t ncb) {
     for (int64_t r = R; r < ld; r++) put_scale(scales, fmt, cb * ld + r, 1.0f, 127);
 }
 
-/* 1x128 groups along the columns of X [M, K] (K is the contraction of the
- * forward and dgrad GEMMs).  Output q [M, K] (ld K), scales
- * [K/128][round_up(M,128)].  Requires K % 128 == 0. */
-int oracle_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
-                        uint8_t* q, void* scales, int fmt) {
-  if (M < 0 || K < 0 || K % OR_GROUP != 0 || ldx < K) return -2;
-  int64_t ncb = K / OR_GROUP;
+/* Groups of G (128, or 32 for MX blocks) along the columns of X [M, K] (K is
+ * the contraction of the forward and dgrad GEMMs).  Output q [M, K] (ld K),
+ * scales [K/G][round_up(M,128)].  Requires K % G == 0. */
+int oracle_quantize_act_g(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                          uint8_t* q, void* scales, int fmt, int G) {
+  if ((G != 128 && G != 32) || M < 0 || K < 0 || K % G != 0 || ldx < K) return -2;
+  int64_t ncb = K / G;
   int64_t lds = round_up128(M);
 #pragma omp parallel for schedule(static)
   for (int64_t r = 0; r < M; r++) {
     float v[OR_GROUP];
     uint8_t c[OR_GROUP];
     for (int64_t g = 0; g < ncb; g++) {
-      for (int j = 0; j < OR_GROUP; j++) v[j] = bf16_to_f32(x[r * ldx + g * OR_GROUP + j]);
+      for (int j = 0; j < G; j++) v[j] = bf16_to_f32(x[r * ldx + g * G + j]);
       float s32 = 0.0f;
       uint8_t e8 = 0;
-      quantize_group(v, OR_GROUP, fmt, c, &s32, &e8);
-      for (int j = 0; j < OR_GROUP; j++) q[r * K + g * OR_GROUP + j] = c[j];
+      quantize_group(v, G, fmt, c, &s32, &e8);
+      for (int j = 0; j < G; j++) q[r * K + g * G + j] = c[j];
       put_scale(scales, fmt, g * lds + r, s32, e8);
     }
   }
@@ -197,30 +201,40 @@ int oracle_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
   return 0;
 }
 
-/* 1x128 groups along the rows (tokens) of X [M, K], i.e. the act quantizer
+int oracle_quantize_act(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                        uint8_t* q, void* scales, int fmt) {
+  return oracle_quantize_act_g(x, M, K, ldx, q, scales, fmt, OR_GROUP);
+}
+
+/* Groups of G along the rows (tokens) of X [M, K], i.e. the act quantizer
  * applied to X^T, as the weight-gradient GEMM contracts over tokens.
- * Output qt [K, M] (ld M), scales [M/128][round_up(K,128)].
+ * Output qt [K, M] (ld M), scales [M/G][round_up(K,128)].
  * Requires M % 128 == 0. */
-int oracle_quantize_act_t(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
-                          uint8_t* qt, void* scales, int fmt) {
-  if (M < 0 || K < 0 || M % OR_GROUP != 0 || ldx < K) return -2;
-  int64_t ncb = M / OR_GROUP;
+int oracle_quantize_act_t_g(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                            uint8_t* qt, void* scales, int fmt, int G) {
+  if ((G != 128 && G != 32) || M < 0 || K < 0 || M % OR_GROUP != 0 || ldx < K) return -2;
+  int64_t ncb = M / G;
   int64_t lds = round_up128(K);
 #pragma omp parallel for schedule(static)
   for (int64_t c = 0; c < K; c++) {
     float v[OR_GROUP];
     uint8_t cd[OR_GROUP];
     for (int64_t g = 0; g < ncb; g++) {
-      for (int j = 0; j < OR_GROUP; j++) v[j] = bf16_to_f32(x[(g * OR_GROUP + j) * ldx + c]);
+      for (int j = 0; j < G; j++) v[j] = bf16_to_f32(x[(g * G + j) * ldx + c]);
       float s32 = 0.0f;
       uint8_t e8 = 0;
-      quantize_group(v, OR_GROUP, fmt, cd, &s32, &e8);
-      for (int j = 0; j < OR_GROUP; j++) qt[c * M + g * OR_GROUP + j] = cd[j];
+      quantize_group(v, G, fmt, cd, &s32, &e8);
+      for (int j = 0; j < G; j++) qt[c * M + g * G + j] = cd[j];
       put_scale(scales, fmt, g * lds + c, s32, e8);
     }
   }
   fill_row_pad(scales, fmt, K, ncb);
   return 0;
+}
+
+int oracle_quantize_act_t(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                          uint8_t* qt, void* scales, int fmt) {
+  return oracle_quantize_act_t_g(x, M, K, ldx, qt, scales, fmt, OR_GROUP);
 }
 
 /* 128x128 blocks of W [N, K]; blocks at the row edge (N % 128 != 0) cover the
@@ -260,8 +274,9 @@ int oracle_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
 
 /* A quantized operand seen as a logical matrix [rows, C] with contraction C:
  *   element (r, k) is q[r*ld + k] when k_major, else q[k*ld + r];
- *   its scale is scales[(k/128)*s_stride_k + t*s_stride_r], where t = r for
- *   1x128 row groups and t = r/128 for 128x128 blocks. */
+ *   its scale is scales[(k/G)*s_stride_k + t*s_stride_r], where t = r for
+ *   row groups and t = r/128 for 128x128 blocks, and G = 32 for 1x32 row
+ *   groups, 128 otherwise. */
 typedef struct {
   const uint8_t* q;
   int64_t ld;
@@ -276,8 +291,9 @@ typedef struct {
 
 static double dequant(const oracle_operand* op, int64_t r, int64_t k) {
   uint8_t c = op->k_major ? op->q[r * op->ld + k] : op->q[k * op->ld + r];
-  int64_t t = (op->gran == OR_GRAN_ROW) ? r : r / OR_GROUP;
-  int64_t si = (k / OR_GROUP) * op->s_stride_k + t * op->s_stride_r;
+  int64_t t = (op->gran == OR_GRAN_BLOCK) ? r / OR_GROUP : r;
+  int64_t g = (op->gran == OR_GRAN_ROW32) ? 32 : OR_GROUP;
+  int64_t si = (k / g) * op->s_stride_k + t * op->s_stride_r;
   double s = (op->fmt == OR_SCALE_FP32) ? (double)((const float*)op->scales)[si]
                                         : ldexp(1.0, (int)((const uint8_t*)op->scales)[si] - 127);
   return oracle_e4m3_decode(c) * s;

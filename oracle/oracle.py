@@ -17,6 +17,7 @@ SCALE_FP32 = 0
 SCALE_UE8M0 = 1
 GRAN_ROW = 0
 GRAN_BLOCK = 1
+GRAN_ROW32 = 2  # 1x32 row groups (MX blocks)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "fp8bq_oracle.c")
@@ -63,6 +64,9 @@ def lib():
         for name in ("oracle_quantize_act", "oracle_quantize_act_t", "oracle_quantize_weight"):
             getattr(L, name).restype = ctypes.c_int
             getattr(L, name).argtypes = qargs
+        for name in ("oracle_quantize_act_g", "oracle_quantize_act_t_g"):
+            getattr(L, name).restype = ctypes.c_int
+            getattr(L, name).argtypes = qargs + [ctypes.c_int]
         L.oracle_gemm.restype = None
         L.oracle_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), ctypes.c_int64,
                                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
@@ -104,25 +108,26 @@ def _scale_dtype(fmt: int):
     return np.float32 if fmt == SCALE_FP32 else np.uint8
 
 
-def quantize_act(x_bits: np.ndarray, fmt: int = SCALE_FP32):
-    """X [M,K] bf16 bits -> (q [M,K] uint8, scales [K/128, round_up(M,128)])."""
+def quantize_act(x_bits: np.ndarray, fmt: int = SCALE_FP32, group: int = 128):
+    """X [M,K] bf16 bits -> (q [M,K] uint8, scales [K/group, round_up(M,128)]);
+    group 128 (the pages' activation groups) or 32 (MX blocks)."""
     x = _as_u16(x_bits)
     M, K = x.shape
     q = np.empty((M, K), np.uint8)
-    s = np.empty((K // 128, row_scale_ld(M)), _scale_dtype(fmt))
-    rc = lib().oracle_quantize_act(x.ctypes.data, M, K, K, q.ctypes.data, s.ctypes.data, fmt)
+    s = np.empty((K // group, row_scale_ld(M)), _scale_dtype(fmt))
+    rc = lib().oracle_quantize_act_g(x.ctypes.data, M, K, K, q.ctypes.data, s.ctypes.data, fmt, group)
     if rc != 0:
         raise ValueError(f"oracle_quantize_act: bad shape ({M},{K})")
     return q, s
 
 
-def quantize_act_t(x_bits: np.ndarray, fmt: int = SCALE_FP32):
-    """X [M,K] bf16 bits -> (qt [K,M] uint8, scales [M/128, round_up(K,128)])."""
+def quantize_act_t(x_bits: np.ndarray, fmt: int = SCALE_FP32, group: int = 128):
+    """X [M,K] bf16 bits -> (qt [K,M] uint8, scales [M/group, round_up(K,128)])."""
     x = _as_u16(x_bits)
     M, K = x.shape
     q = np.empty((K, M), np.uint8)
-    s = np.empty((M // 128, row_scale_ld(K)), _scale_dtype(fmt))
-    rc = lib().oracle_quantize_act_t(x.ctypes.data, M, K, K, q.ctypes.data, s.ctypes.data, fmt)
+    s = np.empty((M // group, row_scale_ld(K)), _scale_dtype(fmt))
+    rc = lib().oracle_quantize_act_t_g(x.ctypes.data, M, K, K, q.ctypes.data, s.ctypes.data, fmt, group)
     if rc != 0:
         raise ValueError(f"oracle_quantize_act_t: bad shape ({M},{K})")
     return q, s
@@ -167,9 +172,9 @@ class Operand:
                          self.fmt, 0, self.s_stride_k, self.s_stride_r)
 
 
-def row_operand(q: np.ndarray, scales: np.ndarray, fmt: int) -> Operand:
-    """Output of quantize_act / quantize_act_t: k-major codes, 1x128 row groups."""
-    return Operand(q, True, GRAN_ROW, scales, fmt, scales.shape[1], 1)
+def row_operand(q: np.ndarray, scales: np.ndarray, fmt: int, group: int = 128) -> Operand:
+    """Output of quantize_act / quantize_act_t: k-major codes, 1x128 (or 1x32) row groups."""
+    return Operand(q, True, GRAN_ROW if group == 128 else GRAN_ROW32, scales, fmt, scales.shape[1], 1)
 
 
 def block_operand(q: np.ndarray, scales: np.ndarray, fmt: int, transposed: bool = False) -> Operand:
