@@ -21,9 +21,10 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "Fp8bqError", "lib", "lib_path",
-    "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_weight", "Operand",
-    "row_operand", "block_operand", "bf16_operand", "gemm", "linear_forward", "linear_dgrad",
+    "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
+    "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
+    "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "Operand",
+    "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "linear_forward", "linear_dgrad",
     "linear_wgrad", "check",
 ]
 
@@ -31,6 +32,7 @@ SCALE_FP32 = 0
 SCALE_UE8M0 = 1
 GRAN_ROW = 0
 GRAN_BLOCK = 1
+GRAN_ROW32 = 2  # MX blocks: 1x32 row groups, UE8M0 scales
 _E4M3 = 0
 _BF16 = 1
 
@@ -78,6 +80,11 @@ def lib():
             f.argtypes = [vp, i64, i64, i64, vp, vp, i32, vp]
         L.fp8bq_quantize_act_dual.restype = i32
         L.fp8bq_quantize_act_dual.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, i32, vp]
+        for name in ("fp8bq_quantize_act_mx", "fp8bq_quantize_act_t_mx"):
+            getattr(L, name).restype = i32
+            getattr(L, name).argtypes = [vp, i64, i64, i64, vp, vp, vp]
+        L.fp8bq_quantize_act_dual_mx.restype = i32
+        L.fp8bq_quantize_act_dual_mx.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.fp8bq_gemm.restype = i32
         L.fp8bq_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
                                  i64, i64, ctypes.c_uint32, vp]
@@ -181,6 +188,41 @@ def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None, qt
     return q, s, qt, st
 
 
+def quantize_act_mx(x: torch.Tensor, q=None, s=None):
+    """X [M,K] bf16 -> (q [M,K], UE8M0 scales [K/32, round_up(M,128)]): 1x32 MX blocks."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = _out(q, (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(s, (K // 32, row_scale_ld(M)), torch.uint8, x.device)
+    _raise(lib().fp8bq_quantize_act_mx(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), _stream(x)),
+           "fp8bq_quantize_act_mx")
+    return q, s
+
+
+def quantize_act_t_mx(x: torch.Tensor, q=None, s=None):
+    """X [M,K] bf16 -> (qt [K,M], UE8M0 scales [M/32, round_up(K,128)]): 1x32 MX blocks along M."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = _out(q, (K, M), torch.float8_e4m3fn, x.device)
+    s = _out(s, (M // 32, row_scale_ld(K)), torch.uint8, x.device)
+    _raise(lib().fp8bq_quantize_act_t_mx(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(), _stream(x)),
+           "fp8bq_quantize_act_t_mx")
+    return q, s
+
+
+def quantize_act_dual_mx(x: torch.Tensor, q=None, s=None, qt=None, st=None):
+    """Both MX layouts of X from one read: (q, s, qt, st) as quantize_act_mx and quantize_act_t_mx."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    q = _out(q, (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(s, (K // 32, row_scale_ld(M)), torch.uint8, x.device)
+    qt = _out(qt, (K, M), torch.float8_e4m3fn, x.device)
+    st = _out(st, (M // 32, row_scale_ld(K)), torch.uint8, x.device)
+    _raise(lib().fp8bq_quantize_act_dual_mx(x.data_ptr(), M, K, x.stride(0), q.data_ptr(), s.data_ptr(),
+                                            qt.data_ptr(), st.data_ptr(), _stream(x)), "fp8bq_quantize_act_dual_mx")
+    return q, s, qt, st
+
+
 def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     """W [N,K] bf16 -> (q [N,K] float8_e4m3fn, scales [K/128, ceil(N/128)])."""
     _check_bf16(w, "w")
@@ -222,6 +264,11 @@ class Operand:
 def row_operand(q: torch.Tensor, scales: torch.Tensor, fmt: int) -> Operand:
     """Codes + scales from quantize_act / quantize_act_t (1x128 row groups)."""
     return Operand(q, True, GRAN_ROW, scales, fmt, scales.shape[1], 1)
+
+
+def mx_operand(q: torch.Tensor, scales: torch.Tensor) -> Operand:
+    """Codes + scales from quantize_act_mx / quantize_act_t_mx (1x32 MX blocks)."""
+    return Operand(q, True, GRAN_ROW32, scales, SCALE_UE8M0, scales.shape[1], 1)
 
 
 def block_operand(q: torch.Tensor, scales: torch.Tensor, fmt: int, transposed: bool = False) -> Operand:

@@ -54,7 +54,8 @@ int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a,
                     fp8bq::GemmOperand* out) {
   if (!op || !op->data) return FP8BQ_ERR_INVALID_ARG;
   if (op->dtype != FP8BQ_E4M3 && op->dtype != FP8BQ_BF16) return FP8BQ_ERR_INVALID_ARG;
-  if (op->gran != FP8BQ_GRAN_ROW_1x128 && op->gran != FP8BQ_GRAN_BLOCK_128x128)
+  if (op->gran != FP8BQ_GRAN_ROW_1x128 && op->gran != FP8BQ_GRAN_BLOCK_128x128 &&
+      op->gran != FP8BQ_GRAN_ROW_1x32)
     return FP8BQ_ERR_INVALID_ARG;
   if (op->fmt != fmt) return FP8BQ_ERR_UNSUPPORTED;
   if (op->k_major != 0 && op->k_major != 1) return FP8BQ_ERR_INVALID_ARG;
@@ -67,7 +68,8 @@ int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a,
   if (!bf16) {
     if (!op->scales) return FP8BQ_ERR_INVALID_ARG;
     if (!aligned16(op->scales)) return FP8BQ_ERR_ALIGN;
-    if (op->gran == FP8BQ_GRAN_ROW_1x128) {
+    if (op->gran == FP8BQ_GRAN_ROW_1x32 && fmt != FP8BQ_SCALE_UE8M0) return FP8BQ_ERR_UNSUPPORTED;
+    if (op->gran == FP8BQ_GRAN_ROW_1x128 || op->gran == FP8BQ_GRAN_ROW_1x32) {
       if (!op->k_major) return FP8BQ_ERR_UNSUPPORTED;
       if (op->s_stride_r != 1 || op->s_stride_k % 128 != 0 || op->s_stride_k < rows)
         return FP8BQ_ERR_SHAPE;
@@ -87,7 +89,8 @@ int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a,
   out->bf16 = bf16;
   out->k_major = op->k_major != 0;
   out->scales = op->scales;
-  out->row_groups = op->gran == FP8BQ_GRAN_ROW_1x128;
+  out->row_groups = op->gran == FP8BQ_GRAN_ROW_1x128 || op->gran == FP8BQ_GRAN_ROW_1x32;
+  out->mx = op->gran == FP8BQ_GRAN_ROW_1x32;
   out->s_stride_k = op->s_stride_k;
   out->s_stride_r = op->s_stride_r;
   return FP8BQ_OK;
@@ -104,7 +107,7 @@ int fp8bq_quantize_act(const void* x, int64_t M, int64_t K, int64_t ldx, void* q
   if (K % 128 != 0) return FP8BQ_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, nullptr, nullptr, fmt,
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, nullptr, nullptr, fmt, 128,
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -116,7 +119,7 @@ int fp8bq_quantize_act_t(const void* x, int64_t M, int64_t K, int64_t ldx, void*
   if (K % 8 != 0) return FP8BQ_ERR_ALIGN;
   if (M == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, nullptr, nullptr, qt, scales, fmt,
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, nullptr, nullptr, qt, scales, fmt, 128,
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -129,7 +132,43 @@ int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, vo
   if (K % 128 != 0 || M % 128 != 0) return FP8BQ_ERR_SHAPE;
   if (M == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, qt, scales_t, fmt,
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, qt, scales_t, fmt, 128,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fp8bq_quantize_act_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                          fp8bq_stream_t stream) {
+  int st = check_quant_args(x, M, K, ldx, q, scales, FP8BQ_SCALE_UE8M0);
+  if (st != FP8BQ_OK) return st;
+  if (K % 128 != 0) return FP8BQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, nullptr, nullptr, FP8BQ_SCALE_UE8M0, 32,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fp8bq_quantize_act_t_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt, void* scales,
+                            fp8bq_stream_t stream) {
+  int st = check_quant_args(x, M, K, ldx, qt, scales, FP8BQ_SCALE_UE8M0);
+  if (st != FP8BQ_OK) return st;
+  if (M % 128 != 0) return FP8BQ_ERR_SHAPE;
+  if (K % 8 != 0) return FP8BQ_ERR_ALIGN;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, nullptr, nullptr, qt, scales, FP8BQ_SCALE_UE8M0, 32,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fp8bq_quantize_act_dual_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                               void* qt, void* scales_t, fp8bq_stream_t stream) {
+  int st = check_quant_args(x, M, K, ldx, q, scales, FP8BQ_SCALE_UE8M0);
+  if (st != FP8BQ_OK) return st;
+  st = check_quant_args(x, M, K, ldx, qt, scales_t, FP8BQ_SCALE_UE8M0);
+  if (st != FP8BQ_OK) return st;
+  if (K % 128 != 0 || M % 128 != 0) return FP8BQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_quant_tiles(x, M, K, ldx, q, scales, qt, scales_t, FP8BQ_SCALE_UE8M0, 32,
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -157,6 +196,7 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
   if (st != FP8BQ_OK) return st;
   st = convert_operand(B, N, K, false, A->fmt, &p.b);
   if (st != FP8BQ_OK) return st;
+  if (p.a.mx != p.b.mx) return FP8BQ_ERR_UNSUPPORTED;  // MX blocks on both operands or neither
   if ((st = device_ok()) != FP8BQ_OK) return st;
   p.d = D;
   p.M = M;
@@ -177,6 +217,8 @@ int64_t fp8bq_scales_bytes(int gran, int fmt, int64_t rows, int64_t contraction)
   const int64_t esz = fmt == FP8BQ_SCALE_FP32 ? 4 : 1;
   const int64_t nkb = contraction / 128;
   if (gran == FP8BQ_GRAN_ROW_1x128) return nkb * fp8bq::round_up128(rows) * esz;
+  if (gran == FP8BQ_GRAN_ROW_1x32)
+    return fmt == FP8BQ_SCALE_UE8M0 ? (contraction / 32) * fp8bq::round_up128(rows) : -1;
   if (gran == FP8BQ_GRAN_BLOCK_128x128) return nkb * ((rows + 127) / 128) * esz;
   return -1;
 }

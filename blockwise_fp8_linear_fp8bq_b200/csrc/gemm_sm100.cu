@@ -595,6 +595,8 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   constexpr bool kFp32 = (FMT == kFmtFp32);
+  constexpr bool kMx = (FMT == kFmtMx);  // 1x32 scales: four per 128-long K block
+  constexpr int kSub = kMx ? 4 : 1;      // scale rows per K block
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
@@ -679,9 +681,16 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tma_load_2d_pair(sb, &p.tmB, fb, brow, kb * BK);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
-          mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz : 0u) + b_sc_bytes);
-          if (a_sc) bulk_load(smem_u32(slot + kSlotRawA), ga + kb * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
-          if (B_ROW) bulk_load(smem_u32(slot + kSlotRawB), gb + kb * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
+          mbar_arrive_expect_tx(fullsc_bar(s), kSub * ((a_sc ? 128u * esz : 0u) + b_sc_bytes));
+#pragma unroll
+          for (int t = 0; t < kSub; ++t) {
+            // scale row kSub * kb + t; MX: the four 32-long sub-blocks of the K block
+            const int64_t sr = static_cast<int64_t>(kSub) * kb + t;
+            if (a_sc)
+              bulk_load(smem_u32(slot + kSlotRawA + 128 * t), ga + sr * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
+            if (B_ROW)
+              bulk_load(smem_u32(slot + kSlotRawB + 256 * t), gb + sr * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
+          }
         }
         __syncwarp();
       }
@@ -729,10 +738,14 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
               const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
               const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
                                               : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
+              // MX: byte k4 of each scale word holds sub-block k4's scale
+              // (scale-factor IDs: A at bits 29-30, B at bits 4-5)
+              const uint32_t idk = kMx ? (idesc | (static_cast<uint32_t>(k4) << 29) | (static_cast<uint32_t>(k4) << 4))
+                                       : idesc;
               if (kFp32)
-                mma_f8_pair(d, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+                mma_f8_pair(d, adesc, bdesc, idk, k4 > 0 ? 1u : 0u);
               else
-                mma_mxf8_pair(d, adesc, bdesc, idesc, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+                mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
             }
             tc_commit_pair(empty_bar(s), 0x3);
             if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
@@ -796,22 +809,29 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(sfready_bar(s));
         } else {
+          // a row's scale word: the one scale replicated (1x128 groups, any
+          // byte selects it), or MX: the four sub-block scales, byte t = t-th
+          auto word = [&](const uint8_t* raw, int stride, int i) -> uint32_t {
+            if (!kMx) return static_cast<uint32_t>(raw[i]) * 0x01010101u;
+            return static_cast<uint32_t>(raw[i]) | (static_cast<uint32_t>(raw[stride + i]) << 8) |
+                   (static_cast<uint32_t>(raw[2 * stride + i]) << 16) | (static_cast<uint32_t>(raw[3 * stride + i]) << 24);
+          };
           const uint8_t* ra = slot + kSlotRawA;
           uint4 wa;
-          wa.x = static_cast<uint32_t>(ra[lane]) * 0x01010101u;
-          wa.y = static_cast<uint32_t>(ra[32 + lane]) * 0x01010101u;
-          wa.z = static_cast<uint32_t>(ra[64 + lane]) * 0x01010101u;
-          wa.w = static_cast<uint32_t>(ra[96 + lane]) * 0x01010101u;
+          wa.x = word(ra, 128, lane);
+          wa.y = word(ra, 128, 32 + lane);
+          wa.z = word(ra, 128, 64 + lane);
+          wa.w = word(ra, 128, 96 + lane);
           *reinterpret_cast<uint4*>(slot + kSlotTm + 16 * lane) = wa;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint4 wb;
             if (B_ROW) {
               const uint8_t* rb = slot + kSlotRawB + 128 * h;
-              wb.x = static_cast<uint32_t>(rb[lane]) * 0x01010101u;
-              wb.y = static_cast<uint32_t>(rb[32 + lane]) * 0x01010101u;
-              wb.z = static_cast<uint32_t>(rb[64 + lane]) * 0x01010101u;
-              wb.w = static_cast<uint32_t>(rb[96 + lane]) * 0x01010101u;
+              wb.x = word(rb, 256, lane);
+              wb.y = word(rb, 256, 32 + lane);
+              wb.z = word(rb, 256, 64 + lane);
+              wb.w = word(rb, 256, 96 + lane);
             } else {
               const uint32_t v = (h == 0 ? b0 : b1) * 0x01010101u;
               wb = make_uint4(v, v, v, v);
@@ -1510,7 +1530,12 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   // BF16 A (fused quantize-on-load), runs CTA pairs (256 x 256 tiles, 128 rows
   // of A and of B per CTA).
   const bool fused = pr.a.bf16;
-  const bool pair = fused || pr.M > 128;
+  const bool mx = pr.a.mx;  // 1x32 blocks on both operands (checked at the ABI)
+  if (mx && (fused || !pr.b.mx || !pr.b.k_major || !pr.b.row_groups)) {
+    *unsupported = true;
+    return cudaSuccess;
+  }
+  const bool pair = fused || mx || pr.M > 128;
   Params prm;
   memset(&prm, 0, sizeof(prm));
   if (fused) {
@@ -1579,6 +1604,7 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
     if (!bk && !br) return launch_fused_variant<kFmtUe8m0, false, false>(prm, di, 4, stream);
     return launch_fused_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
   }
+  if (mx) return launch_pair_variant<kFmtMx, true, true>(prm, di, 6, stream);
   if (pair) {
     if (fp32) {
       if (bk && !br) return launch_pair_variant<kFmtFp32, true, false>(prm, di, 0, stream);

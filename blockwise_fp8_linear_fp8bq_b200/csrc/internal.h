@@ -13,9 +13,10 @@ inline int64_t round_up128(int64_t r) { return (r + 127) / 128 * 128; }
 cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q,
                                 void* scales, int fmt, cudaStream_t stream);
 // TMA-fed activation quantizer: row-group codes (q != nullptr), token-group
-// codes (qt != nullptr), or both from one read of X.
+// codes (qt != nullptr), or both from one read of X; groups of `group` = 128
+// or (UE8M0 only) 32 values.
 cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
-                               void* qt, void* s_cols, int fmt, cudaStream_t stream);
+                               void* qt, void* s_cols, int fmt, int group, cudaStream_t stream);
 
 // Driver entry point of cuTensorMapEncodeTiled (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
@@ -31,7 +32,8 @@ struct GemmOperand {
   bool bf16;     // operand A given as BF16 (quantized inside the GEMM)
   bool k_major;  // contraction contiguous
   const void* scales;
-  bool row_groups;  // 1x128 row groups (else 128x128 blocks)
+  bool row_groups;  // 1x128 (or, with mx, 1x32) row groups, else 128x128 blocks
+  bool mx;          // 1x32 row groups (MX blocks, UE8M0)
   int64_t s_stride_k;
   int64_t s_stride_r;
 };

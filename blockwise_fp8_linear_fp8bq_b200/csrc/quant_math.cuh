@@ -17,6 +17,7 @@ namespace fp8bq {
 
 constexpr int kFmtFp32 = 0;
 constexpr int kFmtUe8m0 = 1;
+constexpr int kFmtMx = 2;  // GEMM only: UE8M0 scales on 1x32 blocks (MX)
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }

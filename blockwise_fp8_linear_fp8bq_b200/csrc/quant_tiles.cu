@@ -65,7 +65,7 @@ __device__ __forceinline__ uint32_t tile_chunk(int r, int c) {
 
 // Row groups: warp w, half-warp h, lane l16 own rows 8 w + 2 i + h (i < 4),
 // chunk l16 (8 values); the amax is a 16-lane reduction.
-template <int FMT>
+template <int FMT, int G>
 __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
                                           int lane) {
   const int half = lane >> 4;
@@ -76,15 +76,15 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   for (int i = 0; i < 4; ++i) {
     const int r = 8 * warp + 2 * i + half;
     v[i] = ld_shared_v4(base + tile_chunk(r, l16));
-    // packed |max| of the 8 values, reduced over the 16 lanes of the row
+    // packed |max| of the 8 values, reduced over the G / 8 lanes of the group
     uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w));
 #pragma unroll
-    for (int o = 8; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    for (int o = G / 16; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
     m2 &= 0x7FFF7FFFu;
     m[i] = fmaxf(bf16_lo(m2), bf16_hi(m2));
   }
   GroupScale gs[4];
-  if constexpr (FMT == kFmtFp32) {
+  if constexpr (FMT == kFmtFp32 && G == 128) {
     // one scale per group, computed by lane 2 i + h and fetched by the others
     float mine = 0.0f;
 #pragma unroll
@@ -110,14 +110,17 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   }
   const int64_t r0 = m0 + 8 * warp + half;
   uint8_t* qrow = p.q + r0 * p.K + k0 + 8 * l16;
+  // the first lane of each group stores its scale: scales [K/G][lds_m]
+  const bool lead = (l16 & (G / 8 - 1)) == 0;
+  const int64_t sg = k0 / G + (l16 * 8) / G;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t r = r0 + 2 * i;
     if (r < p.M) {
       *reinterpret_cast<uint2*>(qrow + 2 * i * p.K) = c[i];
-      if (l16 == 0) store_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r, gs[i]);
-    } else if (r < p.lds_m && l16 == 0) {
-      store_neutral_scale<FMT>(p.s_rows, (k0 >> 7) * p.lds_m + r);
+      if (lead) store_scale<FMT>(p.s_rows, sg * p.lds_m + r, gs[i]);
+    } else if (r < p.lds_m && lead) {
+      store_neutral_scale<FMT>(p.s_rows, sg * p.lds_m + r);
     }
   }
 }
@@ -146,7 +149,7 @@ __device__ __forceinline__ uint4 rotate_bytes_up(const uint4& r, int j) {
 // hit 32 banks.  The codes come out in that rotated order and are rotated
 // back before each lane stores its 16 consecutive tokens (8 lanes: one
 // 128-byte row segment of the transposed codes).
-template <int FMT>
+template <int FMT, int G>
 __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
                                           int lane) {
   const int box = warp & 1;
@@ -166,12 +169,12 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
 #pragma unroll
   for (int i = 0; i < 16; ++i) m2 = absmax_bf16x2(m2, w[i]);
 #pragma unroll
-  for (int o = 4; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  for (int o = G / 32; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
   m2 &= 0x7FFF7FFFu;
   const float m0v = bf16_lo(m2), m1v = bf16_hi(m2);
-  // eight groups per warp: lane 2 a' + b computes column b of pair a'
   GroupScale s0, s1;
-  {
+  if constexpr (FMT == kFmtFp32 && G == 128) {
+    // eight groups per warp: lane 2 a' + b computes column b of pair a'
     float mine = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -183,6 +186,9 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
     const GroupScale gmine = make_scale<FMT>(mine);
     s0 = fetch_scale<FMT>(gmine, 2 * a);
     s1 = fetch_scale<FMT>(gmine, 2 * a + 1);
+  } else {
+    s0 = make_scale<FMT>(m0v);
+    s1 = make_scale<FMT>(m1v);
   }
   uint4 wa[2], wb[2];
 #pragma unroll
@@ -211,23 +217,26 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   const uint4 vb = rotate_bytes_up(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), j);
   const int64_t c = k0 + 64 * box + 2 * (4 * chunk + a);
   const int64_t tok = m0 + 16 * j;
-  const int64_t sidx = (m0 >> 7) * p.lds_k + c;
+  // the first lane of each token group stores its scale: scales [M/G][lds_k]
+  const bool lead = (j & (G / 16 - 1)) == 0;
+  const int64_t sidx = (m0 / G + (16 * j) / G) * p.lds_k + c;
   if (c < p.K) {
     *reinterpret_cast<uint4*>(p.qt + c * p.M + tok) = va;
-    if (j == 0) store_scale<FMT>(p.s_cols, sidx, s0);
-  } else if (c < p.lds_k && j == 0) {
+    if (lead) store_scale<FMT>(p.s_cols, sidx, s0);
+  } else if (c < p.lds_k && lead) {
     store_neutral_scale<FMT>(p.s_cols, sidx);
   }
   if (c + 1 < p.K) {
     *reinterpret_cast<uint4*>(p.qt + (c + 1) * p.M + tok) = vb;
-    if (j == 0) store_scale<FMT>(p.s_cols, sidx + 1, s1);
-  } else if (c + 1 < p.lds_k && j == 0) {
+    if (lead) store_scale<FMT>(p.s_cols, sidx + 1, s1);
+  } else if (c + 1 < p.lds_k && lead) {
     store_neutral_scale<FMT>(p.s_cols, sidx + 1);
   }
 }
 
-template <int FMT, bool ROWS, bool COLS>
+template <int FMT, bool ROWS, bool COLS, int G>
 __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_constant__ QParams p) {
+  static_assert(G == 128 || (G == 32 && FMT == kFmtUe8m0), "1x32 groups use UE8M0 scales");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -285,8 +294,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       const int64_t m0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
       const int64_t k0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
       const uint32_t base = smem_u32(smem + s * kQStage);
-      if (ROWS) tile_rows<FMT>(p, base, m0, k0, warp, lane);
-      if (COLS) tile_cols<FMT>(p, base, m0, k0, warp, lane);
+      if (ROWS) tile_rows<FMT, G>(p, base, m0, k0, warp, lane);
+      if (COLS) tile_cols<FMT, G>(p, base, m0, k0, warp, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
     }
@@ -308,9 +317,9 @@ bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64
   return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool ROWS, bool COLS>
+template <int FMT, bool ROWS, bool COLS, int G>
 cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
-  auto kern = quant_tile_kernel<FMT, ROWS, COLS>;
+  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -331,11 +340,12 @@ cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
 
 }  // namespace
 
-// X [M, K] -> any of: row-group codes q [M, K] + scales [K/128][round_up(M,128)]
-// (q != nullptr), token-group codes qt [K, M] + scales [M/128][round_up(K,128)]
-// (qt != nullptr; M % 128 == 0).  K % 128 == 0 when q is requested.
+// X [M, K] -> any of: row-group codes q [M, K] + scales [K/G][round_up(M,128)]
+// (q != nullptr), token-group codes qt [K, M] + scales [M/G][round_up(K,128)]
+// (qt != nullptr; M % 128 == 0), for groups of G = 128 or (UE8M0 only) 32.
+// K % 128 == 0 when q is requested.
 cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
-                               void* qt, void* s_cols, int fmt, cudaStream_t stream) {
+                               void* qt, void* s_cols, int fmt, int group, cudaStream_t stream) {
   QParams prm;
   std::memset(&prm, 0, sizeof(prm));
   if (!encode_x(&prm.tmX, x, M, K, ldx)) return cudaErrorInvalidValue;
@@ -357,14 +367,21 @@ cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx,
   prm.status = status;
   prm.limit_ns = 2000000000ull;
   const bool rows = q != nullptr, cols = qt != nullptr;
-  if (fmt == kFmtFp32) {
-    if (rows && cols) return launch_tiles<kFmtFp32, true, true>(prm, stream);
-    if (rows) return launch_tiles<kFmtFp32, true, false>(prm, stream);
-    return launch_tiles<kFmtFp32, false, true>(prm, stream);
+  if (group == 32) {
+    if (fmt != kFmtUe8m0) return cudaErrorInvalidValue;
+    if (rows && cols) return launch_tiles<kFmtUe8m0, true, true, 32>(prm, stream);
+    if (rows) return launch_tiles<kFmtUe8m0, true, false, 32>(prm, stream);
+    return launch_tiles<kFmtUe8m0, false, true, 32>(prm, stream);
   }
-  if (rows && cols) return launch_tiles<kFmtUe8m0, true, true>(prm, stream);
-  if (rows) return launch_tiles<kFmtUe8m0, true, false>(prm, stream);
-  return launch_tiles<kFmtUe8m0, false, true>(prm, stream);
+  if (group != 128) return cudaErrorInvalidValue;
+  if (fmt == kFmtFp32) {
+    if (rows && cols) return launch_tiles<kFmtFp32, true, true, 128>(prm, stream);
+    if (rows) return launch_tiles<kFmtFp32, true, false, 128>(prm, stream);
+    return launch_tiles<kFmtFp32, false, true, 128>(prm, stream);
+  }
+  if (rows && cols) return launch_tiles<kFmtUe8m0, true, true, 128>(prm, stream);
+  if (rows) return launch_tiles<kFmtUe8m0, true, false, 128>(prm, stream);
+  return launch_tiles<kFmtUe8m0, false, true, 128>(prm, stream);
 }
 
 }  // namespace fp8bq

@@ -26,7 +26,10 @@
  *         scales[cb * fp8bq_row_scale_ld(R) + r], cb = k / 128; the row
  *         stride is R rounded up to a multiple of 128 and the pad entries
  *         r >= R hold the neutral scale (1.0f, or the byte 127);
- *       128x128 blocks of W [N,K]: scales[kb * ceil(N/128) + nb].
+ *       128x128 blocks of W [N,K]: scales[kb * ceil(N/128) + nb];
+       1x32 row groups (MX blocks, the other reading of "MXFP8 on
+         Blackwell": the OCP Microscaling format's 32-value blocks with
+         E8M0 scales): as 1x128 row groups with cb = k / 32.
  *     FP32 scales are `float`; UE8M0 scales are one byte e + 127 meaning 2^e.
  *   - Scale definitions:  FP32: s = fl32(amax / 448) (s = 1 for an all-zero
  *     group), code q = E4M3_RNE_satfinite(fl32(x / s)).  UE8M0: e = the least
@@ -57,7 +60,11 @@ typedef struct CUstream_st* fp8bq_stream_t;
 #define FP8BQ_ERR_TIMEOUT (-6)     /* a bounded wait inside a GEMM kernel expired   */
 
 typedef enum { FP8BQ_SCALE_FP32 = 0, FP8BQ_SCALE_UE8M0 = 1 } fp8bq_scale_fmt;
-typedef enum { FP8BQ_GRAN_ROW_1x128 = 0, FP8BQ_GRAN_BLOCK_128x128 = 1 } fp8bq_gran;
+typedef enum {
+  FP8BQ_GRAN_ROW_1x128 = 0,
+  FP8BQ_GRAN_BLOCK_128x128 = 1,
+  FP8BQ_GRAN_ROW_1x32 = 2 /* MX blocks: 32 consecutive contraction values, UE8M0 only */
+} fp8bq_gran;
 typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
 
 /*
@@ -72,12 +79,15 @@ typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
  *            is accepted for a 128x128-block operand B (the dgrad GEMM reads
  *            W [N,K] as W^T this way, without a transpose pass).
  *   scales   scale array (ignored when dtype is BF16).
- *   gran     FP8BQ_GRAN_ROW_1x128 (A, or B in the weight-gradient GEMM) or
- *            FP8BQ_GRAN_BLOCK_128x128 (B only).
+ *   gran     FP8BQ_GRAN_ROW_1x128 (A, or B in the weight-gradient GEMM),
+ *            FP8BQ_GRAN_BLOCK_128x128 (B only), or FP8BQ_GRAN_ROW_1x32 (MX:
+ *            A and B both, k_major, UE8M0; the weight is quantized in 1x32
+ *            groups along its contraction like an activation).
  *   fmt      FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0; A and B must agree.
  *   s_stride_k, s_stride_r
- *            the scale of element (r, k) is scales[(k/128)*s_stride_k +
- *            t*s_stride_r], t = r (row groups) or t = r/128 (blocks).  Row
+ *            the scale of element (r, k) is scales[(k/G)*s_stride_k +
+ *            t*s_stride_r], t = r (row groups) or t = r/128 (blocks), G = 32
+ *            for FP8BQ_GRAN_ROW_1x32 and 128 otherwise.  Row
  *            groups need s_stride_r == 1 and s_stride_k a multiple of 128;
  *            blocks are either (ceil(rows/128), 1) or, for W^T, (1, C/128).
  */
@@ -135,6 +145,28 @@ int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, vo
                             void* qt, void* scales_t, int fmt, fp8bq_stream_t stream);
 
 /*
+ * MX-block quantization (1x32 groups, UE8M0 scales): the other reading of
+ * "MXFP8 on Blackwell" ("方法"), with the OCP Microscaling format's 32-value
+ * blocks in place of the 1x128 groups.  Same definitions as the calls above
+ * with 32 for 128; the scale format is always UE8M0.
+ *   fp8bq_quantize_act_mx:    x [M, K] -> q [M, K] (ld K), scales
+ *                             [K/32][fp8bq_row_scale_ld(M)] (bytes); K % 128 == 0.
+ *   fp8bq_quantize_act_t_mx:  x [M, K] -> qt [K, M] (ld M), scales
+ *                             [M/32][fp8bq_row_scale_ld(K)]; M % 128 == 0, K % 8 == 0.
+ *   fp8bq_quantize_act_dual_mx: both, from one read; K % 128 == 0, M % 128 == 0.
+ * A weight W [N, K] takes fp8bq_quantize_act_mx for the forward GEMM and
+ * fp8bq_quantize_act_t_mx (groups along N) for the data-gradient GEMM, since
+ * 1x32 blocks, unlike 128x128 ones, depend on the orientation.
+ * Errors: as fp8bq_quantize_act / _act_t / _act_dual.
+ */
+int fp8bq_quantize_act_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                          fp8bq_stream_t stream);
+int fp8bq_quantize_act_t_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* qt, void* scales,
+                            fp8bq_stream_t stream);
+int fp8bq_quantize_act_dual_mx(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* scales,
+                               void* qt, void* scales_t, fp8bq_stream_t stream);
+
+/*
  * 128x128 weight-block quantization ("方法": weights in 128x128 blocks).
  *   w       BF16 [N, K], leading dimension ldw (ldw >= K, ldw % 8 == 0).
  *   q       E4M3 [N, K], leading dimension K.
@@ -162,7 +194,8 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
  * Errors: ERR_INVALID_ARG, ERR_SHAPE (M,N <= 0, K % 128 != 0, N % 8 != 0),
  * ERR_ALIGN (a pointer not 16-B aligned, a leading dimension not a multiple
  * of 16 bytes), ERR_UNSUPPORTED (mixed scale formats, BF16 B, row-group B
- * that is not k-major), ERR_CUDA (tensor-map encoding or launch failed).
+ * that is not k-major, MX operands mixed with other granularities or not
+ * both k-major UE8M0), ERR_CUDA (tensor-map encoding or launch failed).
  */
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream);
@@ -171,7 +204,8 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
 int64_t fp8bq_row_scale_ld(int64_t rows);
 
 /* Bytes of the scale array for an operand with `rows` rows and contraction
- * `contraction` (a multiple of 128); -1 on bad arguments. */
+ * `contraction` (a multiple of 128); -1 on bad arguments (including
+ * FP8BQ_GRAN_ROW_1x32 with FP32 scales). */
 int64_t fp8bq_scales_bytes(int gran, int fmt, int64_t rows, int64_t contraction);
 
 /*

@@ -97,6 +97,35 @@ def test_dual_quantizer_argument_checks(L):
     assert f(P, 0, 128, 128, P, P, P, P, 0, None) == OK        # empty: no launch
 
 
+@pytest.mark.parametrize("fn", ["fp8bq_quantize_act_mx", "fp8bq_quantize_act_t_mx"])
+def test_mx_quantizer_argument_checks(L, fn):
+    f = getattr(L, fn)
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p]
+    assert f(None, 128, 128, 128, P, P, None) == INVALID
+    assert f(P, 128, 128, 128, None, P, None) == INVALID
+    assert f(P, -1, 128, 128, P, P, None) == SHAPE
+    assert f(P + 8, 128, 128, 128, P, P, None) == ALIGN
+    if fn == "fp8bq_quantize_act_t_mx":
+        assert f(P, 96, 128, 128, P, P, None) == SHAPE   # tokens % 128
+    else:
+        assert f(P, 128, 96, 128, P, P, None) == SHAPE   # columns % 128
+    assert f(P, 0, 128, 128, P, P, None) == OK
+
+
+def test_mx_scale_sizes_and_gemm_checks(L):
+    assert L.fp8bq_scales_bytes(2, 1, 200, 512) == (512 // 32) * 256
+    assert L.fp8bq_scales_bytes(2, 0, 200, 512) == -1  # MX blocks are UE8M0 only
+    out = ctypes.c_void_p(P)
+    mx = dict(gran=2, fmt=1, s_stride_k=256, s_stride_r=1)
+    # MX with FP32 scales, and MX mixed with 1x128 groups, are not built
+    assert L.fp8bq_gemm(ctypes.byref(_op(L, gran=2)), ctypes.byref(_op(L, gran=2)), out, 256, 256, 512, 256, 0,
+                        None) == UNSUPPORTED
+    assert L.fp8bq_gemm(ctypes.byref(_op(L, **mx)), ctypes.byref(_op(L, fmt=1)), out, 256, 256, 512, 256, 0,
+                        None) == UNSUPPORTED
+
+
 def _op(L, **kw):
     import blockwise_fp8_linear_fp8bq_b200 as fp
     d = dict(data=P, ld=512, dtype=0, k_major=1, scales=P, gran=0, fmt=0, s_stride_k=256, s_stride_r=1)
