@@ -134,13 +134,15 @@ class ClockSampler:
 class LayerStep:
     """Device buffers and the launch sequence of one step."""
 
-    def __init__(self, fp, fmt, seed, device, only=None, dual=True):
+    def __init__(self, fp, fmt, seed, device, only=None, dual=True, mx=False):
         self.fp = fp
         self.fmt = fmt
         self.dual = dual
+        self.mx = mx  # 1x32 MX blocks (UE8M0) on every operand; weights quantized in both orientations
         self.items = []
         sdt = torch.float32 if fmt == fp.SCALE_FP32 else torch.uint8
         e4 = torch.float8_e4m3fn
+        g = 32 if mx else 128
         for i, lin in enumerate(linears()):
             if only is not None and lin.name not in only:
                 continue
@@ -149,24 +151,36 @@ class LayerStep:
             it = dict(lin=lin,
                       x=lin.x(s, device=device), w=lin.w(s, device=device), dy=lin.dy(s, device=device),
                       qx=torch.empty(M, K, dtype=e4, device=device),
-                      sx=torch.empty(K // 128, fp.row_scale_ld(M), dtype=sdt, device=device),
+                      sx=torch.empty(K // g, fp.row_scale_ld(M), dtype=sdt, device=device),
                       qw=torch.empty(N, K, dtype=e4, device=device),
-                      sw=torch.empty(K // 128, (N + 127) // 128, dtype=sdt, device=device),
+                      sw=(torch.empty(K // 32, fp.row_scale_ld(N), dtype=sdt, device=device) if mx else
+                          torch.empty(K // 128, (N + 127) // 128, dtype=sdt, device=device)),
                       qd=torch.empty(M, N, dtype=e4, device=device),
-                      sd=torch.empty(N // 128, fp.row_scale_ld(M), dtype=sdt, device=device),
+                      sd=torch.empty(N // g, fp.row_scale_ld(M), dtype=sdt, device=device),
                       qdt=torch.empty(N, M, dtype=e4, device=device),
-                      sdt=torch.empty(M // 128, fp.row_scale_ld(N), dtype=sdt, device=device),
+                      sdt=torch.empty(M // g, fp.row_scale_ld(N), dtype=sdt, device=device),
                       qxt=torch.empty(K, M, dtype=e4, device=device),
-                      sxt=torch.empty(M // 128, fp.row_scale_ld(K), dtype=sdt, device=device),
+                      sxt=torch.empty(M // g, fp.row_scale_ld(K), dtype=sdt, device=device),
                       y=torch.empty(M, N, dtype=torch.bfloat16, device=device),
                       dx=torch.empty(M, K, dtype=torch.bfloat16, device=device),
                       dw=torch.empty(N, K, dtype=torch.bfloat16, device=device))
+            if mx:  # W^T codes grouped along N, for dgrad
+                it["qwt"] = torch.empty(K, N, dtype=e4, device=device)
+                it["swt"] = torch.empty(N // 32, fp.row_scale_ld(K), dtype=sdt, device=device)
             self.items.append(it)
 
     # algorithmic bytes of each quantizer launch (bf16 read, e4m3 write, scales)
     def quant_bytes(self):
         sb = 4 if self.fmt == self.fp.SCALE_FP32 else 1
         tot = 0
+        if self.mx:
+            for it in self.items:
+                lin = it["lin"]
+                M, K, N = lin.M, lin.K, lin.N
+                tot += 2 * (N * K * 3 + N * K // 32)  # W in both orientations
+                tot += M * K * 4 + 2 * M * K // 32     # dual(X)
+                tot += M * N * 4 + 2 * M * N // 32     # dual(dY)
+            return tot
         for it in self.items:
             lin = it["lin"]
             M, K, N = lin.M, lin.K, lin.N
@@ -186,6 +200,8 @@ class LayerStep:
         return sum(3 * it["lin"].flops for it in self.items)
 
     def launches(self):
+        if self.mx:
+            return 7 * len(self.items)
         return (6 if self.dual else 8) * len(self.items)
 
     def run(self, ev=None, external=False):
@@ -205,6 +221,19 @@ class LayerStep:
             b.record()
             ev.append((kind, a, b))
 
+        if self.mx:
+            for it in self.items:
+                timed("quant", lambda: fp.quantize_act_dual_mx(it["x"], it["qx"], it["sx"], it["qxt"], it["sxt"]))
+                timed("quant", lambda: fp.quantize_act_mx(it["w"], it["qw"], it["sw"]))
+                timed("quant", lambda: fp.quantize_act_t_mx(it["w"], it["qwt"], it["swt"]))
+                timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qx"], it["sx"]), fp.mx_operand(it["qw"], it["sw"]),
+                                              it["y"]))
+                timed("quant", lambda: fp.quantize_act_dual_mx(it["dy"], it["qd"], it["sd"], it["qdt"], it["sdt"]))
+                timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]),
+                                              it["dx"]))
+                timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qdt"], it["sdt"]),
+                                              fp.mx_operand(it["qxt"], it["sxt"]), it["dw"]))
+            return
         for it in self.items:
             if self.dual:
                 timed("quant", lambda: fp.quantize_act_dual(it["x"], f, it["qx"], it["sx"], it["qxt"], it["sxt"]))
@@ -236,7 +265,8 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
-    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant)
+    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant,
+                     mx=args.scale == "mx")
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
 
@@ -338,15 +368,21 @@ def run_ours(args, rank, world, dist):
 
 
 # --------------------------------------------------------- oracle on CPU --
-def oracle_sample(seconds_hint: float = 10.0):
+def oracle_format(args):
+    """(scale format, group size) of the oracle sample for --scale."""
+    return {"fp32": (0, 128), "ue8m0": (1, 128), "mx": (1, 32)}[args.scale]
+
+
+def oracle_sample(fmt: int = 0, group: int = 128, size: int = 1):
     """Time the CPU oracle on a bounded sample of the step and extrapolate to
-    the whole step: quantizers on 256-row slabs of each tensor, GEMMs on whole
-    output rows (T rows of each of the 12 GEMMs, T = oracle threads)."""
+    the whole step: quantizers on 256-row slabs of each tensor (x size), GEMMs
+    on whole output rows (size x T rows of each forward GEMM, T = oracle
+    threads)."""
     import numpy as np
     import oracle
     oracle.build()
     T = oracle.num_threads()
-    rows_per_gemm = max(1, T)
+    rows_per_gemm = max(1, T) * size
     q_elems = q_time = 0.0
     g_flops = g_time = 0.0
     full_q_elems = 0
@@ -354,24 +390,32 @@ def oracle_sample(seconds_hint: float = 10.0):
     for i, lin in enumerate(linears()):
         M, K, N = lin.M, lin.K, lin.N
         s = 7000 + 100 * i
-        slab = 256
+        slab = 256 * size
         x = synth.bf16_bits(synth.activations_bf16(slab, K, s))
         w = synth.bf16_bits(synth.weights_bf16(min(N, slab), K, s + 1))
         dy = synth.bf16_bits(synth.grads_bf16(slab, N, s + 2))
         t = time.perf_counter()
-        qx, sx = oracle.quantize_act(x)
-        qw, sw = oracle.quantize_weight(w)
-        qd, sd = oracle.quantize_act(dy)
-        qdt, sdt = oracle.quantize_act_t(dy)
-        qxt, sxt = oracle.quantize_act_t(x)
+        qx, sx = oracle.quantize_act(x, fmt, group)
+        if group == 32:  # MX: the weight in both orientations
+            qw, sw = oracle.quantize_act(w, fmt, group)
+            qwt, swt = oracle.quantize_act_t(synth.bf16_bits(synth.weights_bf16(slab, min(K, slab), s + 5)), fmt, group)
+        else:
+            qw, sw = oracle.quantize_weight(w, fmt)
+        qd, sd = oracle.quantize_act(dy, fmt, group)
+        qdt, sdt = oracle.quantize_act_t(dy, fmt, group)
+        qxt, sxt = oracle.quantize_act_t(x, fmt, group)
         q_time += time.perf_counter() - t
-        q_elems += 2 * x.size + w.size + 2 * dy.size
-        full_q_elems += 2 * M * K + N * K + 2 * M * N
+        q_elems += 2 * x.size + w.size + 2 * dy.size + (slab * min(K, slab) if group == 32 else 0)
+        full_q_elems += 2 * M * K + N * K + 2 * M * N + (N * K if group == 32 else 0)
         # GEMMs: T full output rows of each, operands sized to the real contraction
         xa = synth.bf16_bits(synth.activations_bf16(rows_per_gemm, K, s + 3))
-        qa, sa = oracle.quantize_act(xa)
-        A = oracle.row_operand(qa, sa, 0)
-        B = oracle.block_operand(*oracle.quantize_weight(synth.bf16_bits(synth.weights_bf16(N, K, s + 4))), 0)
+        qa, sa = oracle.quantize_act(xa, fmt, group)
+        A = oracle.row_operand(qa, sa, fmt, group)
+        wb = synth.bf16_bits(synth.weights_bf16(N, K, s + 4))
+        if group == 32:
+            B = oracle.row_operand(*oracle.quantize_act(wb, fmt, group), fmt, group)
+        else:
+            B = oracle.block_operand(*oracle.quantize_weight(wb, fmt), fmt)
         t = time.perf_counter()
         oracle.gemm(A, B)
         g_time += time.perf_counter() - t
@@ -380,7 +424,7 @@ def oracle_sample(seconds_hint: float = 10.0):
     # dgrad and wgrad rows cost the same per FLOP as forward rows in the oracle
     # (one dequantized multiply-add per term), so the forward sample stands for all three
     step_s = full_q_elems * (q_time / q_elems) + full_flops * (g_time / g_flops)
-    sample = (f"4 linears: 256-row slabs through the 3 quantizers and {rows_per_gemm} full output rows "
+    sample = (f"4 linears: {slab}-row slabs through the quantizers and {rows_per_gemm} full output rows "
               f"of each forward GEMM; {q_elems / 1e6:.1f} M quantized elements in {q_time:.2f} s, "
               f"{g_flops / 1e9:.2f} GFLOP in {g_time:.2f} s; extrapolated to the full step")
     return {"step_s": step_s, "tflops": full_flops / step_s / 1e12, "cores": T, "sample": sample,
@@ -394,7 +438,7 @@ def run_reference(args, rank, world):
     t_all = time.perf_counter()
     res = None
     for i in range(args.warmup + args.steps):
-        res = oracle_sample()
+        res = oracle_sample(*oracle_format(args))
         if i >= args.warmup:
             steps.append(res["step_s"])
     step_s = statistics.median(steps) if steps else res["step_s"]
@@ -421,6 +465,25 @@ def case_launchers(step, fp):
     f = fp.SCALE_FP32 if step.fmt == fp.SCALE_FP32 else fp.SCALE_UE8M0
     sb = 4 if f == fp.SCALE_FP32 else 1
     out = {}
+    if step.mx:
+        for it in step.items:
+            lin = it["lin"]
+            M, K, N, n = lin.M, lin.K, lin.N, lin.name
+            out[f"quant_dual_mx:x:{n}"] = ("quant", M * K * 4 + 2 * M * K // 32, lambda it=it: fp.quantize_act_dual_mx(
+                it["x"], it["qx"], it["sx"], it["qxt"], it["sxt"]))
+            out[f"quant_dual_mx:dy:{n}"] = ("quant", M * N * 4 + 2 * M * N // 32, lambda it=it: fp.quantize_act_dual_mx(
+                it["dy"], it["qd"], it["sd"], it["qdt"], it["sdt"]))
+            out[f"quant_act_mx:w:{n}"] = ("quant", N * K * 3 + N * K // 32,
+                                          lambda it=it: fp.quantize_act_mx(it["w"], it["qw"], it["sw"]))
+            out[f"quant_act_t_mx:w:{n}"] = ("quant", N * K * 3 + N * K // 32,
+                                            lambda it=it: fp.quantize_act_t_mx(it["w"], it["qwt"], it["swt"]))
+            out[f"gemm_fwd_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+                fp.mx_operand(it["qx"], it["sx"]), fp.mx_operand(it["qw"], it["sw"]), it["y"]))
+            out[f"gemm_dgrad_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+                fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]), it["dx"]))
+            out[f"gemm_wgrad_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+                fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dw"]))
+        return out
     for it in step.items:
         lin = it["lin"]
         M, K, N, n = lin.M, lin.K, lin.N, lin.name
@@ -462,7 +525,7 @@ def run_case(args):
     torch.cuda.set_device(dev)
     fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
     only = None if args.case == "all" else {args.case.split(":")[-1]}
-    step = LayerStep(fp, fmt, seed=1000, device=dev, only=only)
+    step = LayerStep(fp, fmt, seed=1000, device=dev, only=only, mx=args.scale == "mx")
     step.run()  # produce every operand once
     torch.cuda.synchronize()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -516,8 +579,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--scale", choices=["fp32", "ue8m0"], default="ue8m0",
-                    help="scale format; ue8m0 = the MXFP8 route the pages take on Blackwell")
+    ap.add_argument("--scale", choices=["fp32", "ue8m0", "mx"], default="ue8m0",
+                    help="scale format; ue8m0 = the MXFP8 route the pages take on Blackwell (1x128 groups, "
+                         "128x128 weight blocks); mx = 1x32 MX blocks on every operand")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps eagerly instead of replaying a CUDA graph of the step")
@@ -558,7 +622,8 @@ def main(argv=None):
     e2e_ms = reduce_max(r["e2e"]["ms_per_step"], dist) if r["e2e"] else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample()
+        # a larger sample than each reference-arm step: seconds of CPU work
+        cpu = oracle_sample(*oracle_format(args), size=16)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:

@@ -96,6 +96,8 @@ struct Params {
   CUtensorMap tmA;
   CUtensorMap tmB;
   CUtensorMap tmD;       // BF16 output, 64 x 32 boxes, 128-byte swizzle
+  CUtensorMap tmSA;      // MX only: A's 1x32 scales [K/32][lds_a] bytes, boxes 128 x 4
+  CUtensorMap tmSB;      // MX only: B's 1x32 scales [K/32][lds_b] bytes, boxes 256 x 4
   const void* sA;        // A row-group scales [K/128][lds_a]
   const void* sB;        // B scales (row groups or blocks)
   int64_t sa_stride_k;   // = lds_a
@@ -617,7 +619,8 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < P_STAGES; ++s) {
       // UE8M0: the scale-staging warps of both CTAs also arrive on full[s]
-      mbar_init(full_bar(s), kFp32 ? 1 : 3);
+      // (MX: two staging warps per CTA, one for A's scales, one for B's)
+      mbar_init(full_bar(s), kFp32 ? 1 : (kMx ? 5 : 3));
       mbar_init(fullsc_bar(s), 1);
       mbar_init(empty_bar(s), 1);
       mbar_init(sfready_bar(s), 1);
@@ -648,6 +651,10 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     // Warp-uniform loop; one elected lane issues the copies.
     prefetch_tensormap(&p.tmA);
     prefetch_tensormap(&p.tmB);
+    if (kMx) {
+      prefetch_tensormap(&p.tmSA);
+      prefetch_tensormap(&p.tmSB);
+    }
     uint32_t it = 0;
     bool ok = true;
     for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
@@ -681,15 +688,16 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tma_load_2d_pair(sb, &p.tmB, fb, brow, kb * BK);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
-          mbar_arrive_expect_tx(fullsc_bar(s), kSub * ((a_sc ? 128u * esz : 0u) + b_sc_bytes));
-#pragma unroll
-          for (int t = 0; t < kSub; ++t) {
-            // scale row kSub * kb + t; MX: the four 32-long sub-blocks of the K block
-            const int64_t sr = static_cast<int64_t>(kSub) * kb + t;
-            if (a_sc)
-              bulk_load(smem_u32(slot + kSlotRawA + 128 * t), ga + sr * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
-            if (B_ROW)
-              bulk_load(smem_u32(slot + kSlotRawB + 256 * t), gb + sr * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
+          if (kMx) {
+            // the K block's four 1x32 scale rows of A (128 rows) and of B (256
+            // rows) as two 2-D boxes; past-the-end rows read as zeros
+            mbar_arrive_expect_tx(fullsc_bar(s), 4u * 128u + 4u * 256u);
+            tma_load_2d(smem_u32(slot + kSlotRawA), &p.tmSA, fullsc_bar(s), static_cast<int32_t>(row0), 4 * kb);
+            tma_load_2d(smem_u32(slot + kSlotRawB), &p.tmSB, fullsc_bar(s), nb * P_BN, 4 * kb);
+          } else {
+            mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz : 0u) + b_sc_bytes);
+            if (a_sc) bulk_load(smem_u32(slot + kSlotRawA), ga + kb * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
+            if (B_ROW) bulk_load(smem_u32(slot + kSlotRawB), gb + kb * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
           }
         }
         __syncwarp();
@@ -773,8 +781,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       __syncwarp();
       mbar_wait(final_bar, 0, guard, kTimeoutTeardown);
     }
-  } else if (warp == 2) {
+  } else if (warp == 2 || (kMx && warp == 3)) {
     // ------------------------------------------------------- scale staging
+    // MX: warp 2 stages A's scale words, warp 3 B's (four bytes each).
+    const bool stage_a = !kMx || warp == 2;
+    const bool stage_b = !kMx || warp == 3;
     uint32_t it = 0;
     bool ok = true;
     const uint32_t full_leader_base = mapa_shared(full_bar(0), 0);
@@ -816,15 +827,17 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             return static_cast<uint32_t>(raw[i]) | (static_cast<uint32_t>(raw[stride + i]) << 8) |
                    (static_cast<uint32_t>(raw[2 * stride + i]) << 16) | (static_cast<uint32_t>(raw[3 * stride + i]) << 24);
           };
-          const uint8_t* ra = slot + kSlotRawA;
-          uint4 wa;
-          wa.x = word(ra, 128, lane);
-          wa.y = word(ra, 128, 32 + lane);
-          wa.z = word(ra, 128, 64 + lane);
-          wa.w = word(ra, 128, 96 + lane);
-          *reinterpret_cast<uint4*>(slot + kSlotTm + 16 * lane) = wa;
+          if (stage_a) {
+            const uint8_t* ra = slot + kSlotRawA;
+            uint4 wa;
+            wa.x = word(ra, 128, lane);
+            wa.y = word(ra, 128, 32 + lane);
+            wa.z = word(ra, 128, 64 + lane);
+            wa.w = word(ra, 128, 96 + lane);
+            *reinterpret_cast<uint4*>(slot + kSlotTm + 16 * lane) = wa;
+          }
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < 2 && stage_b; ++h) {
             uint4 wb;
             if (B_ROW) {
               const uint8_t* rb = slot + kSlotRawB + 128 * h;
@@ -1576,6 +1589,25 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.sb_stride_k = pr.b.s_stride_k;
   prm.sb_stride_r = pr.b.s_stride_r;
   prm.sb_len = pr.b.row_groups ? pr.b.s_stride_k : 0;
+  if (mx) {
+    // 1x32 scale arrays as byte matrices [K/32][ld]; boxes of 4 scale rows
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const void* sp[2] = {pr.a.scales, pr.b.scales};
+    const int64_t ld[2] = {pr.a.s_stride_k, pr.b.s_stride_k};
+    const uint32_t boxc[2] = {128, 256};
+    CUtensorMap* maps[2] = {&prm.tmSA, &prm.tmSB};
+    for (int i = 0; i < 2; ++i) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld[i]), static_cast<cuuint64_t>(pr.K / 32)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld[i])};
+      cuuint32_t box[2] = {boxc[i], 4};
+      cuuint32_t es[2] = {1, 1};
+      CUresult r = fn(maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sp[i]), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+  }
   prm.nb_blocks = (pr.N + 127) / 128;
   prm.D = static_cast<uint16_t*>(pr.d);
   prm.ldd = pr.ldd;
