@@ -285,17 +285,24 @@ def bf16_operand(x: torch.Tensor, fmt: int) -> Operand:
     return Operand(x, True, GRAN_ROW, None, fmt, 0, 1, bf16=True)
 
 
-def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """D = deq(A) . deq(B)^T in BF16 ([A.rows, B.rows])."""
+GEMM_ACCUMULATE_F32 = 1
+
+
+def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None, accumulate: bool = False) -> torch.Tensor:
+    """D = deq(A) . deq(B)^T in BF16 ([A.rows, B.rows]); with accumulate=True,
+    `out` is an FP32 [A.rows, B.rows] tensor and the product is added into it."""
     M, N, K = A.rows, B.rows, A.contraction
     if B.contraction != K:
         raise ValueError("contraction mismatch")
-    out = _out(out, (M, N), torch.bfloat16, A.data.device) if out is None else out
-    if out.dtype != torch.bfloat16 or out.dim() != 2 or out.stride(1) != 1 or tuple(out.shape) != (M, N):
-        raise ValueError(f"out must be a row-major bf16 tensor of shape {(M, N)}")
+    dt = torch.float32 if accumulate else torch.bfloat16
+    if accumulate and out is None:
+        raise ValueError("accumulate=True needs the FP32 tensor to add into")
+    out = _out(out, (M, N), dt, A.data.device) if out is None else out
+    if out.dtype != dt or out.dim() != 2 or out.stride(1) != 1 or tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be a row-major {dt} tensor of shape {(M, N)}")
     ca, cb = A._c(), B._c()
-    st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0), 0,
-                          _stream(out))
+    st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0),
+                          GEMM_ACCUMULATE_F32 if accumulate else 0, _stream(out))
     _raise(st, "fp8bq_gemm")
     return out
 

@@ -186,7 +186,8 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream) {
   if (!A || !B || !D) return FP8BQ_ERR_INVALID_ARG;
-  if (flags != 0) return FP8BQ_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<uint32_t>(FP8BQ_GEMM_ACCUMULATE_F32)) != 0) return FP8BQ_ERR_INVALID_ARG;
+  const bool acc = (flags & FP8BQ_GEMM_ACCUMULATE_F32) != 0;
   if (!valid_fmt(A->fmt)) return FP8BQ_ERR_INVALID_ARG;
   if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0 || ldd < N) return FP8BQ_ERR_SHAPE;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BQ_ERR_SHAPE;
@@ -197,6 +198,8 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
   st = convert_operand(B, N, K, false, A->fmt, &p.b);
   if (st != FP8BQ_OK) return st;
   if (p.a.mx != p.b.mx) return FP8BQ_ERR_UNSUPPORTED;  // MX blocks on both operands or neither
+  // FP32 accumulation is built for the weight-gradient layout only
+  if (acc && (p.a.bf16 || !p.a.row_groups || !p.b.row_groups || !p.b.k_major)) return FP8BQ_ERR_UNSUPPORTED;
   if ((st = device_ok()) != FP8BQ_OK) return st;
   p.d = D;
   p.M = M;
@@ -204,6 +207,7 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
   p.K = K;
   p.ldd = ldd;
   p.fmt = A->fmt;
+  p.acc_f32 = acc;
   bool unsupported = false;
   cudaError_t e = fp8bq::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream), &unsupported);
   if (unsupported) return FP8BQ_ERR_UNSUPPORTED;

@@ -209,6 +209,33 @@ __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)
   }
 }
 
+// FP32 accumulation into D (D += tile): the 32 rows x 32 NBOX columns of a
+// warp, as NBOX boxes of 32 x 32 floats (128-byte rows, 128-byte swizzle)
+// through one 4 KB buffer, each added into global memory by a TMA reduce.
+template <int NBOX>
+__device__ __forceinline__ void add_boxes_f32(const Params& p, const float2 (&acc)[16 * NBOX], uint8_t* stage,
+                                              int lane, int m0, int n0) {
+  const uint32_t sbase = smem_u32(stage);
+#pragma unroll
+  for (int j = 0; j < NBOX; ++j) {
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int q = 16 * j + 2 * c;  // float2 index of columns 32 j + 4 c
+      st_shared_v4(sbase + 128 * lane + 16 * (c ^ (lane & 7)), __float_as_uint(acc[q].x), __float_as_uint(acc[q].y),
+                   __float_as_uint(acc[q + 1].x), __float_as_uint(acc[q + 1].y));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int x = n0 + 32 * j;
+      if (x < p.N && m0 < p.M) tma_reduce_add_2d(&p.tmD, sbase, x, m0);
+      bulk_commit_group();
+    }
+  }
+}
+
 template <int FMT, bool B_KMAJOR, bool B_ROW>
 __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant__ Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -581,9 +608,10 @@ struct Cfg {
 };
 }  // namespace pairk
 
-template <int FMT, bool B_KMAJOR, bool B_ROW>
+template <int FMT, bool B_KMAJOR, bool B_ROW, bool ACC = false>
 __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ Params p) {
+  // ACC: D is FP32 and the tile is added into it (D += A B^T), else BF16 D = A B^T
   using pairk::P_BMC;
   using pairk::P_BN;
   using pairk::P_BNC;
@@ -937,7 +965,10 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
-      store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+      if constexpr (ACC)
+        add_boxes_f32<kCols / 32>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+      else
+        store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
     }
     if (lane == 0) bulk_wait_group0();
     __syncwarp();
@@ -1377,8 +1408,8 @@ struct DeviceInfo {
   int sms = 0;
   int* status = nullptr;
   bool attr_set[8] = {};
-  bool pair_attr_set[8] = {};
-  int pair_clusters[8] = {};
+  bool pair_attr_set[12] = {};
+  int pair_clusters[12] = {};
   bool fused_attr_set[8] = {};
   int fused_clusters[8] = {};
 };
@@ -1434,9 +1465,9 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
   return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool BK_, bool BR_>
+template <int FMT, bool BK_, bool BR_, bool ACC_ = false>
 cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cudaStream_t stream) {
-  auto kern = gemm_pair_kernel<FMT, BK_, BR_>;
+  auto kern = gemm_pair_kernel<FMT, BK_, BR_, ACC_>;
   constexpr uint32_t kSmem = pairk::Cfg<FMT == kFmtFp32>::kSmemAlloc;
   if (!di->pair_attr_set[slot]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
@@ -1548,7 +1579,14 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
     *unsupported = true;
     return cudaSuccess;
   }
-  const bool pair = fused || mx || pr.M > 128;
+  // FP32 accumulation (D += A B^T) is built for the weight-gradient layout:
+  // both operands row groups, K-major, on CTA pairs
+  const bool acc = pr.acc_f32;
+  if (acc && (fused || !pr.a.row_groups || !pr.b.row_groups || !pr.b.k_major)) {
+    *unsupported = true;
+    return cudaSuccess;
+  }
+  const bool pair = fused || mx || acc || pr.M > 128;
   Params prm;
   memset(&prm, 0, sizeof(prm));
   if (fused) {
@@ -1574,11 +1612,13 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   {
     auto fn = encode_fn();
     if (!fn) return cudaErrorInvalidValue;
+    // BF16 D: 64 x 32 boxes; FP32 D (accumulating): 32 x 32 boxes; both 128-byte rows
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(pr.N), static_cast<cuuint64_t>(pr.M)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.ldd) * 2};
-    cuuint32_t box[2] = {64, 32};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pr.ldd) * (acc ? 4 : 2)};
+    cuuint32_t box[2] = {acc ? 32u : 64u, 32};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(&prm.tmD, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.d, dims, strides, box, es,
+    CUresult r = fn(&prm.tmD, acc ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, pr.d,
+                    dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -1635,6 +1675,11 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
     if (bk && !br) return launch_fused_variant<kFmtUe8m0, true, false>(prm, di, 3, stream);
     if (!bk && !br) return launch_fused_variant<kFmtUe8m0, false, false>(prm, di, 4, stream);
     return launch_fused_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
+  }
+  if (acc) {
+    if (mx) return launch_pair_variant<kFmtMx, true, true, true>(prm, di, 9, stream);
+    if (fp32) return launch_pair_variant<kFmtFp32, true, true, true>(prm, di, 7, stream);
+    return launch_pair_variant<kFmtUe8m0, true, true, true>(prm, di, 8, stream);
   }
   if (mx) return launch_pair_variant<kFmtMx, true, true>(prm, di, 6, stream);
   if (pair) {

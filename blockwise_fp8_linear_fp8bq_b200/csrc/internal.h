@@ -42,7 +42,8 @@ struct GemmProblem {
   GemmOperand a, b;
   void* d;
   int64_t M, N, K, ldd;
-  int fmt;  // kFmtFp32 / kFmtUe8m0 (both operands)
+  int fmt;        // kFmtFp32 / kFmtUe8m0 (both operands)
+  bool acc_f32;   // D is FP32 and accumulated into (D += A B^T); else BF16 D = A B^T
 };
 
 // Launches the GEMM; returns a cudaError_t (cudaSuccess on success).  Sets

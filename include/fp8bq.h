@@ -67,6 +67,9 @@ typedef enum {
 } fp8bq_gran;
 typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
 
+/* fp8bq_gemm flags */
+#define FP8BQ_GEMM_ACCUMULATE_F32 1u /* D is FP32 and D += A B^T */
+
 /*
  * One GEMM operand, seen as a logical matrix [rows, C] whose second index runs
  * over the contraction C.
@@ -188,9 +191,17 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
  * FP32 scales run the per-128-K promotion path (partial products in tensor
  * memory, rescaled into FP32 accumulators); UE8M0 scales run the block-scaled
  * MMA (MXFP8 route).
- *   D       BF16 [M, N], leading dimension ldd (ldd >= N, ldd % 8 == 0).
+ *   D       BF16 [M, N], leading dimension ldd (ldd >= N, ldd % 8 == 0); FP32
+ *           with FP8BQ_GEMM_ACCUMULATE_F32.
  *   K       contraction length, K % 128 == 0, K > 0.
- *   flags   0 (reserved for future hints; other values give ERR_INVALID_ARG).
+ *   flags   0, or FP8BQ_GEMM_ACCUMULATE_F32: D is then FP32 (ld ldd floats)
+ *           and the product is added into it, D += A B^T, each element
+ *           rounded once from D_old + the FP32 accumulator (the weight
+ *           gradient added into an FP32 master gradient: "方法" keeps master
+ *           weights and optimizer state in FP32).  Built for operands that are
+ *           both row groups (1x128 or 1x32), k_major, E4M3; other
+ *           combinations give ERR_UNSUPPORTED.  Other flag bits give
+ *           ERR_INVALID_ARG.
  * Errors: ERR_INVALID_ARG, ERR_SHAPE (M,N <= 0, K % 128 != 0, N % 8 != 0),
  * ERR_ALIGN (a pointer not 16-B aligned, a leading dimension not a multiple
  * of 16 bytes), ERR_UNSUPPORTED (mixed scale formats, BF16 B, row-group B

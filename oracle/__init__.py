@@ -11,6 +11,7 @@ from .oracle import (  # noqa: F401
     SCALE_UE8M0,
     GRAN_ROW,
     GRAN_BLOCK,
+    GRAN_ROW32,
     build,
     lib,
     num_threads,
@@ -18,6 +19,7 @@ from .oracle import (  # noqa: F401
     e4m3_encode,
     ue8m0_exponent,
     quantize_act,
+    gemm_accumulate,
     quantize_act_t,
     quantize_weight,
     row_scale_ld,

@@ -76,6 +76,20 @@ def lib():
     return _lib
 
 
+def gemm_accumulate(A: "Operand", B: "Operand", d0: np.ndarray, rows=None, cols=None) -> np.ndarray:
+    """float64 d0[rows x cols] + deq(A)[rows] . deq(B)[cols]^T: the weight gradient
+    added into an FP32 master gradient (the Puro-2B digest, section "方法": master
+    weights and optimizer state stay in FP32).  d0 is the FP32 gradient before
+    the call, [A.rows, B.rows]."""
+    g = gemm(A, B, rows, cols)
+    d = np.asarray(d0, np.float64)
+    if rows is not None:
+        d = d[np.asarray(rows, np.int64)]
+    if cols is not None:
+        d = d[:, np.asarray(cols, np.int64)]
+    return d + g
+
+
 def num_threads() -> int:
     return int(lib().oracle_num_threads())
 

@@ -143,7 +143,8 @@ def test_gemm_argument_checks(L):
     assert g(None, B) == INVALID
     assert g(A, None) == INVALID
     assert g(A, B, D=None) == INVALID
-    assert g(A, B, flags=1) == INVALID
+    assert g(A, B, flags=2) == INVALID               # unknown flag bit
+    assert g(A, B, flags=1) == UNSUPPORTED           # FP32 accumulation needs row-group B
     assert g(A, B, k=100) == SHAPE
     assert g(A, B, n=100, ldd=104) == SHAPE          # N % 8
     assert g(A, B, m=0) == SHAPE

@@ -248,3 +248,65 @@ def test_lm_head_forward_full_size(fmt):
     compare_sampled_on_device(D, o_row(qx, sx, fmt), o_block(qw, sw, fmt), "lm_head fwd", seed=4200)
     del D
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------- FP32 accumulation (D += A B^T) --
+@pytest.mark.parametrize("fmt", ["fp32", "ue8m0", "mx"])
+@pytest.mark.parametrize("shape", [(256, 384, 512), (200, 136, 256), (8, 8, 128)])
+def test_wgrad_accumulates_into_fp32(fmt, shape):
+    """dW_master += dY^T X with FP32 D: the master gradient plus the product."""
+    Nr, Kc, Mt = shape  # output rows (N), output columns (K), contraction (tokens, multiple of 128)
+    Mt = max(128, Mt // 128 * 128)
+    dy = synth.grads_bf16(Mt, Nr, seed=51, device="cuda") * 1000
+    x = synth.activations_bf16(Mt, Kc, seed=52, device="cuda")
+    if fmt == "mx":
+        qa, sa = fp.quantize_act_t_mx(dy)
+        qb, sb = fp.quantize_act_t_mx(x)
+        A, B = fp.mx_operand(qa, sa), fp.mx_operand(qb, sb)
+        Ao = oracle.row_operand(u8(qa), sa.cpu().numpy(), 1, group=32)
+        Bo = oracle.row_operand(u8(qb), sb.cpu().numpy(), 1, group=32)
+    else:
+        f = fp.SCALE_FP32 if fmt == "fp32" else fp.SCALE_UE8M0
+        qa, sa = fp.quantize_act_t(dy, f)
+        qb, sb = fp.quantize_act_t(x, f)
+        A, B = fp.row_operand(qa, sa, f), fp.row_operand(qb, sb, f)
+        Ao, Bo = o_row(qa, sa, f), o_row(qb, sb, f)
+    d0 = torch.randn(Nr, Kc, device="cuda", dtype=torch.float32, generator=torch.Generator("cuda").manual_seed(53))
+    D = d0.clone()
+    fp.gemm(A, B, D, accumulate=True)
+    torch.cuda.synchronize()
+    got = D.cpu().numpy().astype(np.float64)
+    ref = oracle.gemm_accumulate(Ao, Bo, d0.cpu().numpy())
+    # FP32 output: the product's error (FP32 accumulation) plus one FP32 rounding of the sum
+    diff = got - ref
+    prod = ref - d0.cpu().numpy().astype(np.float64)
+    rms = np.sqrt(np.mean(prod * prod))
+    assert np.linalg.norm(diff) <= 5e-3 * np.linalg.norm(prod), fmt
+    assert np.all(np.abs(diff) <= 1e-3 * rms + np.abs(ref) * 2.0 ** -23), fmt
+
+
+def test_wgrad_accumulate_full_size_gate_up():
+    """dW of gate/up (12288 x 2048, contraction 16384) added into an FP32 master
+    gradient, UE8M0 scales; sampled rows and columns against the oracle."""
+    lin = synth.GATE_UP
+    x = lin.x(4300, device="cuda")
+    dy = lin.dy(4300, device="cuda")
+    f = fp.SCALE_UE8M0
+    qa, sa = fp.quantize_act_t(dy, f)
+    qb, sb = fp.quantize_act_t(x, f)
+    del x, dy
+    d0 = torch.randn(lin.N, lin.K, device="cuda", dtype=torch.float32, generator=torch.Generator("cuda").manual_seed(54))
+    D = d0.clone()
+    fp.gemm(fp.row_operand(qa, sa, f), fp.row_operand(qb, sb, f), D, accumulate=True)
+    torch.cuda.synchronize()
+    rows = sample_indices(lin.N, 4, 55)
+    cols = sample_indices(lin.K, 4, 56)
+    Ao, Bo = o_row(qa, sa, f), o_row(qb, sb, f)
+    d0h = d0.cpu().numpy()
+    got = np.concatenate([D[torch.from_numpy(rows).cuda(), :].cpu().numpy().astype(np.float64).ravel(),
+                          D[:, torch.from_numpy(cols).cuda()].cpu().numpy().astype(np.float64).ravel()])
+    ref = np.concatenate([oracle.gemm_accumulate(Ao, Bo, d0h, rows=rows).ravel(),
+                          oracle.gemm_accumulate(Ao, Bo, d0h, cols=cols).ravel()])
+    prod = ref - np.concatenate([d0h[rows].astype(np.float64).ravel(), d0h[:, cols].astype(np.float64).ravel()])
+    diff = got - ref
+    assert np.linalg.norm(diff) <= 5e-3 * np.linalg.norm(prod)

@@ -128,3 +128,25 @@ def test_sampled_rows_and_cols_match_full(oracle_lib):
     assert np.array_equal(oracle_lib.gemm(A, B, rows=r, cols=c), full[np.ix_(r, c)])
     assert np.array_equal(oracle_lib.gemm(A, B, rows=r), full[r])
     assert np.array_equal(oracle_lib.gemm(A, B, cols=c), full[:, c])
+
+
+def test_gemm_accumulate_adds_the_product_to_the_master_gradient():
+    """gemm_accumulate(A, B, d0) = d0 + deq(A) deq(B)^T, against numpy on
+    torch-decoded operands, on all and on selected rows/columns."""
+    import oracle as orc
+    from test_oracle_quant import bits_of, dec, make_input, scale_value
+    M, N, K = 256, 136, 256
+    a = make_input(M, K, seed=41)
+    b = make_input(N, K, seed=42)
+    qa, sa = orc.quantize_act(bits_of(a), 0)
+    qb, sb = orc.quantize_act(bits_of(b), 0)
+    d0 = np.random.default_rng(43).standard_normal((M, N)).astype(np.float32)
+    A, B = orc.row_operand(qa, sa, 0), orc.row_operand(qb, sb, 0)
+    ra = dec(qa) * np.repeat(scale_value(sa, 0)[:, :M].T, 128, axis=1)
+    rb = dec(qb) * np.repeat(scale_value(sb, 0)[:, :N].T, 128, axis=1)
+    ref = d0.astype(np.float64) + ra @ rb.T
+    got = orc.gemm_accumulate(A, B, d0)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-10)
+    rows, cols = np.array([0, 7, 255]), np.array([3, 135])
+    assert np.allclose(orc.gemm_accumulate(A, B, d0, rows=rows, cols=cols), ref[np.ix_(rows, cols)], rtol=1e-12,
+                       atol=1e-10)
