@@ -20,6 +20,7 @@ from .oracle import (  # noqa: F401
     ue8m0_exponent,
     quantize_act,
     gemm_accumulate,
+    swiglu,
     quantize_act_t,
     quantize_weight,
     row_scale_ld,

@@ -270,6 +270,49 @@ int oracle_quantize_weight(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
   return 0;
 }
 
+/* ---------------------------------------------- SwiGLU (the producer op) -- */
+
+/* Round a double to the nearest bfloat16, ties to even, in one step (no
+ * intermediate float), keeping the sign of zero.  bf16 keeps 8 significant
+ * bits with fp32's exponent range (subnormal quantum 2^-133). */
+static uint16_t f64_to_bf16_rne(double v) {
+  uint16_t sign = signbit(v) ? 0x8000 : 0;
+  double a = fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  frexp(a, &e); /* a = m 2^e, m in [0.5, 1) */
+  int E = e - 1;
+  if (E < -126) E = -126;
+  double quantum = ldexp(1.0, E - 7);
+  double n = a / quantum; /* exact: power-of-two scaling */
+  double fl = floor(n);
+  double rem = n - fl;
+  if (rem > 0.5 || (rem == 0.5 && fmod(fl, 2.0) == 1.0)) fl += 1.0;
+  float f = (float)(fl * quantum); /* <= 9 significant bits: exact in float */
+  uint32_t u;
+  memcpy(&u, &f, 4);
+  return (uint16_t)(sign | (u >> 16));
+}
+
+/* The down projection's input: SwiGLU of the fused gate/up output.  gu is
+ * BF16 [M, 2F] holding [gate | up] (the gate/up GEMM's two halves side by
+ * side); h[r][c] = silu(g) * u with silu(g) = g / (1 + e^-g), g = gu[r][c],
+ * u = gu[r][F + c], evaluated in float64 (h64, optional) and rounded once to
+ * bfloat16 (h, ld F): the activation the layer stores in BF16 ("清华开源
+ * Puro-2B", section "精度": activations outside the FP8 matmuls stay BF16). */
+void oracle_swiglu(const uint16_t* gu, int64_t M, int64_t F, int64_t ld, uint16_t* h, double* h64) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < M; r++) {
+    for (int64_t c = 0; c < F; c++) {
+      double g = (double)bf16_to_f32(gu[r * ld + c]);
+      double u = (double)bf16_to_f32(gu[r * ld + F + c]);
+      double v = g / (1.0 + exp(-g)) * u;
+      if (h64) h64[r * F + c] = v;
+      h[r * F + c] = f64_to_bf16_rne(v);
+    }
+  }
+}
+
 /* ------------------------------------------------------------------ GEMM -- */
 
 /* A quantized operand seen as a logical matrix [rows, C] with contraction C:

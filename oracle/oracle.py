@@ -72,8 +72,23 @@ def lib():
                                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
                                   ctypes.c_void_p]
         L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_swiglu.restype = None
+        L.oracle_swiglu.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                    ctypes.c_void_p, ctypes.c_void_p]
         _lib = L
     return _lib
+
+
+def swiglu(gu_bits: np.ndarray, with_f64: bool = False):
+    """[gate | up] BF16 bits [M, 2F] -> h BF16 bits [M, F] = RNE_bf16(silu(g) u),
+    evaluated in float64 (and the float64 values when with_f64)."""
+    gu = _as_u16(gu_bits)
+    M, F2 = gu.shape
+    F = F2 // 2
+    h = np.empty((M, F), np.uint16)
+    h64 = np.empty((M, F), np.float64) if with_f64 else None
+    lib().oracle_swiglu(gu.ctypes.data, M, F, F2, h.ctypes.data, h64.ctypes.data if with_f64 else None)
+    return (h, h64) if with_f64 else h
 
 
 def gemm_accumulate(A: "Operand", B: "Operand", d0: np.ndarray, rows=None, cols=None) -> np.ndarray:
