@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
     "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
-    "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "Operand",
+    "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "Operand",
     "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "linear_forward", "linear_dgrad",
     "linear_wgrad", "check",
 ]
@@ -83,6 +83,8 @@ def lib():
         for name in ("fp8bq_quantize_act_mx", "fp8bq_quantize_act_t_mx"):
             getattr(L, name).restype = i32
             getattr(L, name).argtypes = [vp, i64, i64, i64, vp, vp, vp]
+        L.fp8bq_swiglu_quantize.restype = i32
+        L.fp8bq_swiglu_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
         L.fp8bq_quantize_act_dual_mx.restype = i32
         L.fp8bq_quantize_act_dual_mx.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.fp8bq_gemm.restype = i32
@@ -186,6 +188,25 @@ def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None, qt
                                        qt.data_ptr(), st.data_ptr(), fmt, _stream(x))
     _raise(rc, "fp8bq_quantize_act_dual")
     return q, s, qt, st
+
+
+def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = True, keep_h: bool = False):
+    """[gate | up] bf16 [M, 2F] -> (q, s, qt, st, h): h = silu(gate) * up in BF16
+    quantized as quantize_act (q, s) and, with transposed, quantize_act_t (qt, st);
+    h itself is returned when keep_h (else None), qt/st are None without transposed."""
+    _check_bf16(gu, "gu")
+    M, F2 = gu.shape
+    F = F2 // 2
+    q = _out(None, (M, F), torch.float8_e4m3fn, gu.device)
+    s = _out(None, (F // 128, row_scale_ld(M)), _scale_dtype(fmt), gu.device)
+    qt = _out(None, (F, M), torch.float8_e4m3fn, gu.device) if transposed else None
+    st = _out(None, (M // 128, row_scale_ld(F)), _scale_dtype(fmt), gu.device) if transposed else None
+    h = _out(None, (M, F), torch.bfloat16, gu.device) if keep_h else None
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    rc = lib().fp8bq_swiglu_quantize(gu.data_ptr(), M, F, gu.stride(0), ptr(h), q.data_ptr(), s.data_ptr(),
+                                     ptr(qt), ptr(st), fmt, _stream(gu))
+    _raise(rc, "fp8bq_swiglu_quantize")
+    return q, s, qt, st, h
 
 
 def quantize_act_mx(x: torch.Tensor, q=None, s=None):

@@ -172,6 +172,20 @@ int fp8bq_quantize_act_dual_mx(const void* x, int64_t M, int64_t K, int64_t ldx,
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int fp8bq_swiglu_quantize(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* scales,
+                          void* qt, void* scales_t, int fmt, fp8bq_stream_t stream) {
+  int st = check_quant_args(gu, M, 2 * F, ldgu, q, scales, fmt);
+  if (st != FP8BQ_OK) return st;
+  if ((qt == nullptr) != (scales_t == nullptr)) return FP8BQ_ERR_INVALID_ARG;
+  if (qt != nullptr && (!aligned16(qt) || !aligned16(scales_t))) return FP8BQ_ERR_ALIGN;
+  if (h != nullptr && !aligned16(h)) return FP8BQ_ERR_ALIGN;
+  if (F % 128 != 0 || (qt != nullptr && M % 128 != 0)) return FP8BQ_ERR_SHAPE;
+  if (M == 0 || F == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_swiglu_quant(gu, M, F, ldgu, h, q, scales, qt, scales_t, fmt,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, void* scales,
                           int fmt, fp8bq_stream_t stream) {
   int st = check_quant_args(w, N, K, ldw, q, scales, fmt);

@@ -18,6 +18,11 @@ cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw
 cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
                                void* qt, void* s_cols, int fmt, int group, cudaStream_t stream);
 
+// SwiGLU of [gate | up] fused with the quantization of its output h
+// (row groups, and token groups when qt != nullptr); h optionally stored.
+cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* s_rows,
+                                void* qt, void* s_cols, int fmt, cudaStream_t stream);
+
 // Driver entry point of cuTensorMapEncodeTiled (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Multiprocessor count of the current device (cached).

@@ -34,11 +34,19 @@ constexpr int kQConsumers = 16;                 // consumer warps 0..15; warp 16
 constexpr int kQThreads = 32 * (kQConsumers + 1);
 constexpr uint32_t kQBox = 128 * 128;           // 64 bf16 columns x 128 rows: 16 KB
 constexpr uint32_t kQStage = 2 * kQBox;
-constexpr uint32_t kQOffBar = kQStages * kQStage;
-constexpr uint32_t kQNumBars = 2 * kQStages;  // full[S], empty[S]
-constexpr uint32_t kQOffMisc = kQOffBar + kQNumBars * 8;
-constexpr uint32_t kQSmem = kQOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
-static_assert(kQSmem <= 232448, "shared memory budget");
+// Shared-memory layout.  SW (SwiGLU producer fused in): a stage holds the
+// gate tile and the up tile (64 KB), three stages, and an h-ready barrier
+// per stage; otherwise one 32 KB tile a stage, six stages.
+template <bool SW>
+struct QCfg {
+  static constexpr int kStages = SW ? 3 : kQStages;
+  static constexpr uint32_t kStage = SW ? 2 * kQStage : kQStage;
+  static constexpr uint32_t kOffBar = kStages * kStage;
+  static constexpr uint32_t kNumBars = 3 * kStages;  // full[S], empty[S], hready[S]
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kSmem = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmem <= 232448, "shared memory budget");
+};
 
 constexpr int kQTimeoutProducer = 11;
 constexpr int kQTimeoutConsumer = 12;
@@ -55,7 +63,27 @@ struct QParams {
   int tiles_k, num_tiles;
   int* status;
   uint64_t limit_ns;
+  // SwiGLU producer: X is h = silu(gate) * up of tmX's [gate | up] columns
+  int64_t up_off;   // column of up[0] (= F)
+  uint16_t* h;      // optional BF16 h [M, K] (ld ldh) written on the way
+  int64_t ldh;
 };
+
+// h = silu(g) u = g u / (1 + e^-g) in fp32 (IEEE division, full-precision
+// exponential), rounded to bf16 (nearest, ties to even; finite values).
+__device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const float g = k ? bf16_hi(g2) : bf16_lo(g2);
+    const float u = k ? bf16_hi(u2) : bf16_lo(u2);
+    const float h = __fdiv_rn(g * u, 1.0f + expf(-g));
+    const uint32_t b = __float_as_uint(h);
+    const uint32_t r = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
+    out |= r << (16 * k);
+  }
+  return out;
+}
 
 // Byte offset of 16-byte chunk c (0..15, 8 bf16 each) of tile row r: chunks
 // 0..7 in the first box, 8..15 in the second; 128-byte swizzle within a box.
@@ -234,24 +262,28 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   }
 }
 
-template <int FMT, bool ROWS, bool COLS, int G>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW>
 __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_constant__ QParams p) {
   static_assert(G == 128 || (G == 32 && FMT == kFmtUe8m0), "1x32 groups use UE8M0 scales");
+  using C = QCfg<SW>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kQOffBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
-  auto empty_bar = [&](int s) { return smem_u32(&bars[kQStages + s]); };
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kQOffMisc);
+  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
+  auto hready_bar = [&](int s) { return smem_u32(&bars[2 * S + s]); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), kQConsumers);
+      mbar_init(hready_bar(s), kQConsumers);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -264,36 +296,66 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kQStages;
-      const uint32_t ph = (it / kQStages) & 1;
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kQTimeoutProducer))) { ok = false; break; }
       if (elect_one()) {
         const int32_t m0 = (tile / p.tiles_k) * 128;
         const int32_t k0 = (tile % p.tiles_k) * 128;
-        // a box wholly past K (ragged K, COLS only) is not loaded: its
-        // columns are never stored and form groups of their own
-        const bool second = k0 + 64 < p.K;
-        const uint32_t dst = smem_u32(smem + s * kQStage);
-        mbar_arrive_expect_tx(full_bar(s), second ? kQStage : kQBox);
-        tma_load_2d(dst, &p.tmX, full_bar(s), k0, m0);
-        if (second) tma_load_2d(dst + kQBox, &p.tmX, full_bar(s), k0 + 64, m0);
+        const uint32_t dst = smem_u32(smem + s * C::kStage);
+        if (SW) {
+          // gate columns k0 .. k0 + 127 and up columns F + k0 .. (F % 128 == 0)
+          const int32_t u0 = static_cast<int32_t>(p.up_off) + k0;
+          mbar_arrive_expect_tx(full_bar(s), 2 * kQStage);
+          tma_load_2d(dst, &p.tmX, full_bar(s), k0, m0);
+          tma_load_2d(dst + kQBox, &p.tmX, full_bar(s), k0 + 64, m0);
+          tma_load_2d(dst + kQStage, &p.tmX, full_bar(s), u0, m0);
+          tma_load_2d(dst + kQStage + kQBox, &p.tmX, full_bar(s), u0 + 64, m0);
+        } else {
+          // a box wholly past K (ragged K, COLS only) is not loaded: its
+          // columns are never stored and form groups of their own
+          const bool second = k0 + 64 < p.K;
+          mbar_arrive_expect_tx(full_bar(s), second ? kQStage : kQBox);
+          tma_load_2d(dst, &p.tmX, full_bar(s), k0, m0);
+          if (second) tma_load_2d(dst + kQBox, &p.tmX, full_bar(s), k0 + 64, m0);
+        }
       }
       __syncwarp();
     }
     // teardown: every load issued has landed before the CTA exits
     const uint32_t total = it;
-    for (uint32_t j = (total > kQStages ? total - kQStages : 0); j < total; ++j)
-      mbar_wait(full_bar(j % kQStages), (j / kQStages) & 1, guard, kQTimeoutProducer);
+    for (uint32_t j = (total > S ? total - S : 0); j < total; ++j)
+      mbar_wait(full_bar(j % S), (j / S) & 1, guard, kQTimeoutProducer);
   } else {
     // ------------------------------------------------------------ consumers
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
-      const int s = it % kQStages;
-      const uint32_t ph = (it / kQStages) & 1;
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kQTimeoutConsumer))) break;
       const int64_t m0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
       const int64_t k0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
-      const uint32_t base = smem_u32(smem + s * kQStage);
+      const uint32_t base = smem_u32(smem + s * C::kStage);
+      if constexpr (SW) {
+        // h over the gate tile, in place: thread t takes chunk t % 16 of rows
+        // t / 16 + 32 i (the same swizzled offset in both tiles)
+        const int t = threadIdx.x;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = t / 16 + 32 * i;
+          const uint32_t off = tile_chunk(r, t % 16);
+          const uint4 g = ld_shared_v4(base + off);
+          const uint4 u = ld_shared_v4(base + kQStage + off);
+          const uint4 h = make_uint4(swiglu_bf16x2(g.x, u.x), swiglu_bf16x2(g.y, u.y), swiglu_bf16x2(g.z, u.z),
+                                     swiglu_bf16x2(g.w, u.w));
+          st_shared_v4(base + off, h.x, h.y, h.z, h.w);
+          if (p.h != nullptr && m0 + r < p.M)
+            *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + k0 + 8 * (t % 16)) = h;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hready_bar(s));
+        if (!__all_sync(0xffffffffu, mbar_wait(hready_bar(s), ph, guard, kQTimeoutConsumer))) break;
+      }
       if (ROWS) tile_rows<FMT, G>(p, base, m0, k0, warp, lane);
       if (COLS) tile_cols<FMT, G>(p, base, m0, k0, warp, lane);
       __syncwarp();
@@ -317,9 +379,10 @@ bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64
   return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool ROWS, bool COLS, int G>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW = false>
 cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
-  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G>;
+  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G, SW>;
+  constexpr uint32_t kQSmem = QCfg<SW>::kSmem;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -382,6 +445,43 @@ cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx,
   if (rows && cols) return launch_tiles<kFmtUe8m0, true, true, 128>(prm, stream);
   if (rows) return launch_tiles<kFmtUe8m0, true, false, 128>(prm, stream);
   return launch_tiles<kFmtUe8m0, false, true, 128>(prm, stream);
+}
+
+// SwiGLU fused with the quantization of its output: gu BF16 [M, 2F] holding
+// [gate | up] -> h = silu(gate) * up (BF16, optionally stored to h [M, F]),
+// quantized as quantize_act (q, s_rows) and, when qt != nullptr, as
+// quantize_act_t (qt, s_cols).  F % 128 == 0; M % 128 == 0 when qt is set.
+cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* s_rows,
+                                void* qt, void* s_cols, int fmt, cudaStream_t stream) {
+  QParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!encode_x(&prm.tmX, gu, M, 2 * F, ldgu)) return cudaErrorInvalidValue;
+  prm.M = M;
+  prm.K = F;
+  prm.q = static_cast<uint8_t*>(q);
+  prm.s_rows = s_rows;
+  prm.lds_m = round_up128(M);
+  prm.qt = static_cast<uint8_t*>(qt);
+  prm.s_cols = s_cols;
+  prm.lds_k = round_up128(F);
+  prm.tiles_k = static_cast<int>(F / 128);
+  const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  prm.num_tiles = static_cast<int>(tiles);
+  prm.up_off = F;
+  prm.h = static_cast<uint16_t*>(h);
+  prm.ldh = F;
+  int* status = nullptr;
+  cudaError_t e = device_status_word(&status);
+  if (e != cudaSuccess) return e;
+  prm.status = status;
+  prm.limit_ns = 2000000000ull;
+  const bool cols = qt != nullptr;
+  if (fmt == kFmtFp32)
+    return cols ? launch_tiles<kFmtFp32, true, true, 128, true>(prm, stream)
+                : launch_tiles<kFmtFp32, true, false, 128, true>(prm, stream);
+  return cols ? launch_tiles<kFmtUe8m0, true, true, 128, true>(prm, stream)
+              : launch_tiles<kFmtUe8m0, true, false, 128, true>(prm, stream);
 }
 
 }  // namespace fp8bq

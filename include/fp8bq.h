@@ -148,6 +148,32 @@ int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, vo
                             void* qt, void* scales_t, int fmt, fp8bq_stream_t stream);
 
 /*
+ * SwiGLU fused with the quantization of its output: the down projection's
+ * input produced and quantized in one pass, without a BF16 round trip
+ * through HBM.  The pages keep the activation function outside the FP8
+ * matmuls ("清华开源 Puro-2B", section "精度"; the digest's "方法": a
+ * Qwen3-1.7B-like model, whose MLP is SwiGLU); this call has no counterpart
+ * on the pages beyond computing that BF16 activation and quantizing it.
+ *   gu        BF16 [M, 2F], leading dimension ldgu: [gate | up], the gate/up
+ *             GEMM's output with the two halves side by side.
+ *   h         optional BF16 [M, F] (ld F): h = silu(gate) * up =
+ *             gate * up / (1 + e^-gate) in FP32, rounded to BF16 (nearest,
+ *             ties to even); may be NULL.  Within one BF16 ulp of the exact
+ *             value.
+ *   q, scales h quantized as fp8bq_quantize_act (1x128 groups along F) of
+ *             exactly that BF16 h: E4M3 [M, F] (ld F), scales
+ *             [F/128][fp8bq_row_scale_ld(M)].
+ *   qt, scales_t  optional (both or neither): h quantized as
+ *             fp8bq_quantize_act_t: [F, M] (ld M), [M/128][fp8bq_row_scale_ld(F)].
+ *   fmt       FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0.
+ * Errors: ERR_INVALID_ARG (null gu, q or scales; only one of qt, scales_t;
+ * bad fmt), ERR_SHAPE (F % 128 != 0; M % 128 != 0 with qt; ldgu < 2F),
+ * ERR_ALIGN (as fp8bq_quantize_act, and h, qt, scales_t 16-B aligned).
+ */
+int fp8bq_swiglu_quantize(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* scales,
+                          void* qt, void* scales_t, int fmt, fp8bq_stream_t stream);
+
+/*
  * MX-block quantization (1x32 groups, UE8M0 scales): the other reading of
  * "MXFP8 on Blackwell" ("方法"), with the OCP Microscaling format's 32-value
  * blocks in place of the 1x128 groups.  Same definitions as the calls above
