@@ -483,6 +483,9 @@ def case_launchers(step, fp):
                 fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]), it["dx"]))
             out[f"gemm_wgrad_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
                 fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dw"]))
+            it["dwf"] = torch.zeros(N, K, dtype=torch.float32, device=it["dw"].device)
+            out[f"gemm_wgrad_acc_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+                fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dwf"], accumulate=True))
         return out
     for it in step.items:
         lin = it["lin"]
@@ -507,6 +510,19 @@ def case_launchers(step, fp):
             fp.row_operand(it["qd"], it["sd"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
         out[f"gemm_wgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+        # the same product added into an FP32 master gradient (D += A B^T)
+        it["dwf"] = torch.zeros(N, K, dtype=torch.float32, device=it["dw"].device)
+        out[f"gemm_wgrad_acc:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
+            fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dwf"],
+            accumulate=True))
+        if n == "down":
+            # the down projection's input from the gate/up output [M, 2K] in one
+            # pass: SwiGLU, then both code layouts (vs a BF16 h written and read back)
+            gen = torch.Generator(device=it["x"].device)
+            gen.manual_seed(977)
+            it["gu"] = torch.randn(M, 2 * K, generator=gen, device=it["x"].device).to(torch.bfloat16)
+            out[f"quant_swiglu:{n}"] = ("quant", M * 2 * K * 2 + 2 * M * K + 2 * (K // 128) * M * sb,
+                                        lambda it=it: fp.swiglu_quantize(it["gu"], f))
         # fused quantize-on-load: BF16 A quantized inside the GEMM
         out[f"gemm_fwd_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))

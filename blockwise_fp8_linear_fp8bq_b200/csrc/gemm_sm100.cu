@@ -223,8 +223,7 @@ __device__ __forceinline__ void add_boxes_f32(const Params& p, const float2 (&ac
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const int q = 16 * j + 2 * c;  // float2 index of columns 32 j + 4 c
-      st_shared_v4(sbase + 128 * lane + 16 * (c ^ (lane & 7)), __float_as_uint(acc[q].x), __float_as_uint(acc[q].y),
-                   __float_as_uint(acc[q + 1].x), __float_as_uint(acc[q + 1].y));
+      st_shared_v4f(sbase + 128 * lane + 16 * (c ^ (lane & 7)), acc[q].x, acc[q].y, acc[q + 1].x, acc[q + 1].y);
     }
     fence_proxy_async_smem();
     __syncwarp();

@@ -69,15 +69,19 @@ struct QParams {
   int64_t ldh;
 };
 
-// h = silu(g) u = g u / (1 + e^-g) in fp32 (IEEE division, full-precision
-// exponential), rounded to bf16 (nearest, ties to even; finite values).
+// h = silu(g) u = g u / (1 + e^-g) in fp32, rounded to bf16 (nearest, ties
+// to even; finite values).  The fast exponential and division keep the fp32
+// value within a few parts in 2^20 of the exact one, far inside the one-bf16-
+// ulp (2^-8) bound the result is specified to: the bf16 rounding hides them
+// except next to a rounding boundary.  For gate < -87, e^-g overflows and
+// h = +-0.
 __device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
   uint32_t out = 0;
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const float g = k ? bf16_hi(g2) : bf16_lo(g2);
     const float u = k ? bf16_hi(u2) : bf16_lo(u2);
-    const float h = __fdiv_rn(g * u, 1.0f + expf(-g));
+    const float h = __fdividef(g * u, 1.0f + __expf(-g));
     const uint32_t b = __float_as_uint(h);
     const uint32_t r = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
     out |= r << (16 * k);
