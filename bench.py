@@ -134,10 +134,12 @@ class ClockSampler:
 class LayerStep:
     """Device buffers and the launch sequence of one step."""
 
-    def __init__(self, fp, fmt, seed, device, only=None, dual=True, mx=False):
+    def __init__(self, fp, fmt, seed, device, only=None, dual=True, mx=False, split=True):
         self.fp = fp
         self.fmt = fmt
         self.dual = dual
+        # GEMM workspace: the last round of output tiles may be split along K
+        self.ws = fp.gemm_workspace(device) if split else None
         self.mx = mx  # 1x32 MX blocks (UE8M0) on every operand; weights quantized in both orientations
         self.items = []
         sdt = torch.float32 if fmt == fp.SCALE_FP32 else torch.uint8
@@ -227,12 +229,12 @@ class LayerStep:
                 timed("quant", lambda: fp.quantize_act_mx(it["w"], it["qw"], it["sw"]))
                 timed("quant", lambda: fp.quantize_act_t_mx(it["w"], it["qwt"], it["swt"]))
                 timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qx"], it["sx"]), fp.mx_operand(it["qw"], it["sw"]),
-                                              it["y"]))
+                                              it["y"], workspace=self.ws))
                 timed("quant", lambda: fp.quantize_act_dual_mx(it["dy"], it["qd"], it["sd"], it["qdt"], it["sdt"]))
                 timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]),
-                                              it["dx"]))
+                                              it["dx"], workspace=self.ws))
                 timed("gemm", lambda: fp.gemm(fp.mx_operand(it["qdt"], it["sdt"]),
-                                              fp.mx_operand(it["qxt"], it["sxt"]), it["dw"]))
+                                              fp.mx_operand(it["qxt"], it["sxt"]), it["dw"], workspace=self.ws))
             return
         for it in self.items:
             if self.dual:
@@ -241,18 +243,19 @@ class LayerStep:
                 timed("quant", lambda: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
             timed("quant", lambda: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qx"], it["sx"], f),
-                                          fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+                                          fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=self.ws))
             if self.dual:
                 timed("quant", lambda: fp.quantize_act_dual(it["dy"], f, it["qd"], it["sd"], it["qdt"], it["sdt"]))
             else:
                 timed("quant", lambda: fp.quantize_act(it["dy"], f, it["qd"], it["sd"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qd"], it["sd"], f),
-                                          fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
+                                          fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"],
+                                          workspace=self.ws))
             if not self.dual:
                 timed("quant", lambda: fp.quantize_act_t(it["dy"], f, it["qdt"], it["sdt"]))
                 timed("quant", lambda: fp.quantize_act_t(it["x"], f, it["qxt"], it["sxt"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qdt"], it["sdt"], f),
-                                          fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+                                          fp.row_operand(it["qxt"], it["sxt"], f), it["dw"], workspace=self.ws))
 
 
 def l2_flush(buf):
@@ -266,7 +269,7 @@ def run_ours(args, rank, world, dist):
     torch.cuda.set_device(dev)
     fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
     step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant,
-                     mx=args.scale == "mx")
+                     mx=args.scale == "mx", split=not args.no_split)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
 
@@ -523,11 +526,11 @@ def case_launchers(step, fp):
             out[f"quant_act_t_mx:w:{n}"] = ("quant", N * K * 3 + N * K // 32,
                                             lambda it=it: fp.quantize_act_t_mx(it["w"], it["qwt"], it["swt"]))
             out[f"gemm_fwd_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-                fp.mx_operand(it["qx"], it["sx"]), fp.mx_operand(it["qw"], it["sw"]), it["y"]))
+                fp.mx_operand(it["qx"], it["sx"]), fp.mx_operand(it["qw"], it["sw"]), it["y"], workspace=step.ws))
             out[f"gemm_dgrad_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-                fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]), it["dx"]))
+                fp.mx_operand(it["qd"], it["sd"]), fp.mx_operand(it["qwt"], it["swt"]), it["dx"], workspace=step.ws))
             out[f"gemm_wgrad_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-                fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dw"]))
+                fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dw"], workspace=step.ws))
             it["dwf"] = torch.zeros(N, K, dtype=torch.float32, device=it["dw"].device)
             out[f"gemm_wgrad_acc_mx:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
                 fp.mx_operand(it["qdt"], it["sdt"]), fp.mx_operand(it["qxt"], it["sxt"]), it["dwf"], accumulate=True))
@@ -550,11 +553,13 @@ def case_launchers(step, fp):
         out[f"quant_dual:dy:{n}"] = ("quant", M * N * 4 + ((N // 128) * M + (M // 128) * N) * sb,
                                      lambda it=it: fp.quantize_act_dual(it["dy"], f, it["qd"], it["sd"], it["qdt"], it["sdt"]))
         out[f"gemm_fwd:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-            fp.row_operand(it["qx"], it["sx"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+            fp.row_operand(it["qx"], it["sx"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=step.ws))
         out[f"gemm_dgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-            fp.row_operand(it["qd"], it["sd"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
+            fp.row_operand(it["qd"], it["sd"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"],
+            workspace=step.ws))
         out[f"gemm_wgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-            fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dw"]))
+            fp.row_operand(it["qdt"], it["sdt"], f), fp.row_operand(it["qxt"], it["sxt"], f), it["dw"],
+            workspace=step.ws))
         # the same product added into an FP32 master gradient (D += A B^T)
         it["dwf"] = torch.zeros(N, K, dtype=torch.float32, device=it["dw"].device)
         out[f"gemm_wgrad_acc:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
@@ -570,9 +575,10 @@ def case_launchers(step, fp):
                                         lambda it=it: fp.swiglu_quantize(it["gu"], f))
         # fused quantize-on-load: BF16 A quantized inside the GEMM
         out[f"gemm_fwd_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-            fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"]))
+            fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=step.ws))
         out[f"gemm_dgrad_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
-            fp.bf16_operand(it["dy"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"]))
+            fp.bf16_operand(it["dy"], f), fp.block_operand(it["qw"], it["sw"], f, transposed=True), it["dx"],
+            workspace=step.ws))
     return out
 
 
@@ -586,7 +592,7 @@ def run_case(args):
     torch.cuda.set_device(dev)
     fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
     only = None if args.case == "all" else {args.case.split(":")[-1]}
-    step = LayerStep(fp, fmt, seed=1000, device=dev, only=only, mx=args.scale == "mx")
+    step = LayerStep(fp, fmt, seed=1000, device=dev, only=only, mx=args.scale == "mx", split=not args.no_split)
     step.run()  # produce every operand once
     torch.cuda.synchronize()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -648,6 +654,8 @@ def main(argv=None):
                     help="launch the timed steps eagerly instead of replaying a CUDA graph of the step")
     ap.add_argument("--separate-quant", action="store_true",
                     help="quantize each activation layout in its own launch instead of the dual pass")
+    ap.add_argument("--no-split", action="store_true",
+                    help="GEMMs without a workspace: no output tiles split along K")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="time single kernels instead of the step: 'all' or a name such as gemm_fwd:gate_up")
@@ -710,6 +718,7 @@ def main(argv=None):
                    "activation_quant": "separate act / act_t launches" if args.separate_quant
                    else "dual (one read of X and of dY, both code layouts)",
                    "launch": "eager" if args.no_graph else "CUDA graph of the timed steps",
+                   "gemm_tiles": "whole tiles" if args.no_split else "last round split along K where it pays",
                    "parallelism": f"replicas{world}", "l2": "flushed between steps (write of 2x L2)"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": gemm_tflops / fp8_peak, "traffic": traffic,

@@ -24,8 +24,8 @@ __all__ = [
     "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
     "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
     "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "Operand",
-    "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "linear_forward", "linear_dgrad",
-    "linear_wgrad", "check",
+    "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "gemm_workspace", "linear_forward",
+    "linear_dgrad", "linear_wgrad", "check",
 ]
 
 SCALE_FP32 = 0
@@ -90,6 +90,11 @@ def lib():
         L.fp8bq_gemm.restype = i32
         L.fp8bq_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
                                  i64, i64, ctypes.c_uint32, vp]
+        L.fp8bq_gemm_ws.restype = i32
+        L.fp8bq_gemm_ws.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
+                                    i64, i64, ctypes.c_uint32, vp, i64, vp]
+        L.fp8bq_gemm_workspace_bytes.restype = i64
+        L.fp8bq_gemm_workspace_bytes.argtypes = []
         L.fp8bq_row_scale_ld.restype = i64
         L.fp8bq_row_scale_ld.argtypes = [i64]
         L.fp8bq_scales_bytes.restype = i64
@@ -309,9 +314,24 @@ def bf16_operand(x: torch.Tensor, fmt: int) -> Operand:
 GEMM_ACCUMULATE_F32 = 1
 
 
-def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None, accumulate: bool = False) -> torch.Tensor:
+def gemm_workspace(device: Optional[torch.device] = None) -> torch.Tensor:
+    """A zeroed workspace for gemm(..., workspace=...) on `device` (uint8,
+    fp8bq_gemm_workspace_bytes() long).  Every completed GEMM leaves its flags
+    zero; GEMMs that may run at the same time need one each."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        n = lib().fp8bq_gemm_workspace_bytes()
+    if n < 0:
+        raise RuntimeError("fp8bq_gemm_workspace_bytes: no usable device")
+    return torch.zeros(n, dtype=torch.uint8, device=dev)
+
+
+def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None, accumulate: bool = False,
+         workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
     """D = deq(A) . deq(B)^T in BF16 ([A.rows, B.rows]); with accumulate=True,
-    `out` is an FP32 [A.rows, B.rows] tensor and the product is added into it."""
+    `out` is an FP32 [A.rows, B.rows] tensor and the product is added into it.
+    With a `workspace` (gemm_workspace()), the last round of output tiles may
+    be split along K over all CTA pairs (fp8bq_gemm_ws)."""
     M, N, K = A.rows, B.rows, A.contraction
     if B.contraction != K:
         raise ValueError("contraction mismatch")
@@ -322,9 +342,17 @@ def gemm(A: Operand, B: Operand, out: Optional[torch.Tensor] = None, accumulate:
     if out.dtype != dt or out.dim() != 2 or out.stride(1) != 1 or tuple(out.shape) != (M, N):
         raise ValueError(f"out must be a row-major {dt} tensor of shape {(M, N)}")
     ca, cb = A._c(), B._c()
-    st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0),
-                          GEMM_ACCUMULATE_F32 if accumulate else 0, _stream(out))
-    _raise(st, "fp8bq_gemm")
+    flags = GEMM_ACCUMULATE_F32 if accumulate else 0
+    if workspace is None:
+        st = lib().fp8bq_gemm(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0), flags,
+                              _stream(out))
+        _raise(st, "fp8bq_gemm")
+        return out
+    if not workspace.is_cuda or workspace.device != out.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the output's device")
+    st = lib().fp8bq_gemm_ws(ctypes.byref(ca), ctypes.byref(cb), out.data_ptr(), M, N, K, out.stride(0), flags,
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(out))
+    _raise(st, "fp8bq_gemm_ws")
     return out
 
 

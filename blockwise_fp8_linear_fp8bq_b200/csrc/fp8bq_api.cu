@@ -199,6 +199,18 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
 
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream) {
+  return fp8bq_gemm_ws(A, B, D, M, N, K, ldd, flags, nullptr, 0, stream);
+}
+
+int64_t fp8bq_gemm_workspace_bytes(void) {
+  if (device_ok() != FP8BQ_OK) return -1;
+  int sms = 0;
+  if (fp8bq::device_sm_count(&sms) != cudaSuccess) return -1;
+  return static_cast<int64_t>(sms / 2) * fp8bq::kWsSlotBytes;
+}
+
+int fp8bq_gemm_ws(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
+                  int64_t ldd, uint32_t flags, void* workspace, int64_t workspace_bytes, fp8bq_stream_t stream) {
   if (!A || !B || !D) return FP8BQ_ERR_INVALID_ARG;
   if ((flags & ~static_cast<uint32_t>(FP8BQ_GEMM_ACCUMULATE_F32)) != 0) return FP8BQ_ERR_INVALID_ARG;
   const bool acc = (flags & FP8BQ_GEMM_ACCUMULATE_F32) != 0;
@@ -206,6 +218,8 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
   if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0 || ldd < N) return FP8BQ_ERR_SHAPE;
   if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BQ_ERR_SHAPE;
   if (!aligned16(D) || ldd % 8 != 0) return FP8BQ_ERR_ALIGN;
+  if (workspace != nullptr && workspace_bytes < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8BQ_ERR_ALIGN;
   fp8bq::GemmProblem p;
   int st = convert_operand(A, M, K, true, A->fmt, &p.a);
   if (st != FP8BQ_OK) return st;
@@ -222,6 +236,8 @@ int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t 
   p.ldd = ldd;
   p.fmt = A->fmt;
   p.acc_f32 = acc;
+  p.ws = workspace;
+  p.ws_bytes = workspace != nullptr ? workspace_bytes : 0;
   bool unsupported = false;
   cudaError_t e = fp8bq::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream), &unsupported);
   if (unsupported) return FP8BQ_ERR_UNSUPPORTED;

@@ -91,6 +91,7 @@ constexpr int kTimeoutMma = 2;
 constexpr int kTimeoutScale = 3;
 constexpr int kTimeoutEpilogue = 4;
 constexpr int kTimeoutTeardown = 5;
+constexpr int kTimeoutSplit = 6;
 
 struct Params {
   CUtensorMap tmA;
@@ -111,7 +112,62 @@ struct Params {
   int num_m, num_n, num_tiles, num_kb;
   int* status;
   uint64_t limit_ns;
+  // Split tiles (CTA-pair kernel, BF16 D): tiles [dp_tiles, num_tiles) are
+  // shared along K by all clusters.  A tile's head piece (from K block 0)
+  // keeps its partial sum; every other piece stores its FP32 partial sum
+  // into the workspace slot of its cluster and raises that slot's flags; the
+  // head piece adds those partials and rounds the tile to BF16 once.
+  // dp_tiles == num_tiles: nothing is split.
+  int dp_tiles;
+  CUtensorMap tmW;  // workspace [clusters * 256][256] FP32, 32 x 32 boxes, 128-byte swizzle
+  float* ws;        // one 256 x 256 partial-sum slot per cluster
+  int* ws_flag;     // per slot and epilogue warp slice: 1 = partial stored (0 between calls)
 };
+
+// ----------------------------------------------------------- work units --
+// A cluster's work: the tiles cl, cl + ncl, ... below dp_tiles, each whole;
+// then its share of the split tiles: their K blocks laid end to end (tile by
+// tile) and cut into ncl ranges of nearly equal length, range c going to
+// cluster c.  A range is shorter than one tile's K extent (the split tiles
+// are fewer than the clusters), so it covers parts of at most two tiles: the
+// tail of one (the cluster's first unit) and the head of the next (its last
+// unit).  Hence a cluster holds at most one piece that does not start at K
+// block 0, and a tile's head piece is the last unit of its cluster.
+struct Unit {
+  int tile;  // < 0: no more work
+  int kb0, kb1;
+  bool split;  // covers only part of the tile's K blocks
+};
+
+__device__ __forceinline__ int64_t split_bound(const Params& p, int c, int ncl) {
+  return static_cast<int64_t>(p.num_tiles - p.dp_tiles) * p.num_kb * c / ncl;
+}
+
+__device__ __forceinline__ Unit split_unit(const Params& p, int64_t g, int c, int ncl) {
+  const int64_t hi = split_bound(p, c + 1, ncl);
+  Unit u{-1, 0, 0, false};
+  if (g >= hi) return u;
+  u.tile = p.dp_tiles + static_cast<int>(g / p.num_kb);
+  u.kb0 = static_cast<int>(g % p.num_kb);
+  const int64_t left = hi - g;
+  u.kb1 = left < p.num_kb - u.kb0 ? u.kb0 + static_cast<int>(left) : p.num_kb;
+  u.split = u.kb1 - u.kb0 < p.num_kb;
+  return u;
+}
+
+__device__ __forceinline__ Unit first_unit(const Params& p, int c, int ncl) {
+  if (c < p.dp_tiles) return Unit{c, 0, p.num_kb, false};
+  return split_unit(p, split_bound(p, c, ncl), c, ncl);
+}
+
+__device__ __forceinline__ Unit next_unit(const Params& p, const Unit& u, int c, int ncl) {
+  if (u.tile < p.dp_tiles) {
+    const int t = u.tile + ncl;
+    if (t < p.dp_tiles) return Unit{t, 0, p.num_kb, false};
+    return split_unit(p, split_bound(p, c, ncl), c, ncl);
+  }
+  return split_unit(p, static_cast<int64_t>(u.tile - p.dp_tiles) * p.num_kb + u.kb1, c, ncl);
+}
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
   const int group = tile / (kGroupM * num_n);
@@ -209,12 +265,36 @@ __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)
   }
 }
 
+// FP32 tile slice stored as is (no accumulation): a split tile's partial sum
+// into the workspace, the boxes and staging of add_boxes_f32.
+template <int NBOX>
+__device__ __forceinline__ void store_boxes_f32(const CUtensorMap* map, const float2 (&acc)[16 * NBOX], uint8_t* stage,
+                                                int lane, int m0, int n0) {
+  const uint32_t sbase = smem_u32(stage);
+#pragma unroll
+  for (int j = 0; j < NBOX; ++j) {
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int q = 16 * j + 2 * c;
+      st_shared_v4f(sbase + 128 * lane + 16 * (c ^ (lane & 7)), acc[q].x, acc[q].y, acc[q + 1].x, acc[q + 1].y);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map, sbase, n0 + 32 * j, m0);
+      bulk_commit_group();
+    }
+  }
+}
+
 // FP32 accumulation into D (D += tile): the 32 rows x 32 NBOX columns of a
 // warp, as NBOX boxes of 32 x 32 floats (128-byte rows, 128-byte swizzle)
 // through one 4 KB buffer, each added into global memory by a TMA reduce.
 template <int NBOX>
-__device__ __forceinline__ void add_boxes_f32(const Params& p, const float2 (&acc)[16 * NBOX], uint8_t* stage,
-                                              int lane, int m0, int n0) {
+__device__ __forceinline__ void add_boxes_f32(const CUtensorMap* map, int xlim, int ylim, const float2 (&acc)[16 * NBOX],
+                                              uint8_t* stage, int lane, int m0, int n0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
   for (int j = 0; j < NBOX; ++j) {
@@ -229,7 +309,7 @@ __device__ __forceinline__ void add_boxes_f32(const Params& p, const float2 (&ac
     __syncwarp();
     if (lane == 0) {
       const int x = n0 + 32 * j;
-      if (x < p.N && m0 < p.M) tma_reduce_add_2d(&p.tmD, sbase, x, m0);
+      if (x < xlim && m0 < ylim) tma_reduce_add_2d(map, sbase, x, m0);
       bulk_commit_group();
     }
   }
@@ -597,8 +677,9 @@ struct Cfg {
   static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
   static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
   static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
-  // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final
-  static constexpr uint32_t kNumBars = 5 * kStages + 5;
+  // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final;
+  // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps)
+  static constexpr uint32_t kNumBars = 5 * kStages + 5 + kEpiWarps;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
@@ -625,7 +706,6 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   constexpr bool kFp32 = (FMT == kFmtFp32);
   constexpr bool kMx = (FMT == kFmtMx);  // 1x32 scales: four per 128-long K block
-  constexpr int kSub = kMx ? 4 : 1;      // scale rows per K block
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
@@ -639,6 +719,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   auto tfull_bar = [&](int b) { return bar(5 * P_STAGES + b); };
   auto tempty_bar = [&](int b) { return bar(5 * P_STAGES + 2 + b); };
   const uint32_t final_bar = bar(5 * P_STAGES + 4);
+  auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 5 + w); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
@@ -658,6 +739,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       mbar_init(tempty_bar(b), 2 * C::kEpiWarps);
     }
     mbar_init(final_bar, 1);
+    for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(eload_bar(w), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -669,7 +751,6 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialized, TMEM of both allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int KB = p.num_kb;
   const int cl = static_cast<int>(cluster_id_x());
   const int ncl = static_cast<int>(nclusters_x());
 
@@ -684,9 +765,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     }
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+    for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
       const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
       const int32_t brow = nb * P_BN + P_BNC * static_cast<int>(rank);
       const uint32_t esz = kFp32 ? 4u : 1u;
@@ -698,7 +779,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       }
       const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + row0 * esz;
       const uint8_t* gb = static_cast<const uint8_t*>(p.sB) + static_cast<int64_t>(nb) * P_BN * esz;
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
         const int s = it % P_STAGES;
         const uint32_t ph = (it / P_STAGES) & 1;
         if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer))) { ok = false; break; }
@@ -745,8 +826,8 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
-      for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
           uint32_t d = tmem_base;
@@ -780,13 +861,13 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
               if (kFp32)
                 mma_f8_pair(d, adesc, bdesc, idk, k4 > 0 ? 1u : 0u);
               else
-                mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > 0 || k4 > 0) ? 1u : 0u);
+                mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > u.kb0 || k4 > 0) ? 1u : 0u);
             }
             tc_commit_pair(empty_bar(s), 0x3);
             if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
           };
-          if (!kFp32 && kb == 0) {
-            // first K block of a tile: the scale factors (own TMEM columns)
+          if (!kFp32 && kb == u.kb0) {
+            // first K block of a tile (or piece): the scale factors (own TMEM columns)
             // are copied while the epilogue still drains the accumulator of
             // the previous tile; the MMAs wait for it
             if (elect_one()) issue_sf();
@@ -816,18 +897,20 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     const uint32_t full_leader_base = mapa_shared(full_bar(0), 0);
-    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
+    for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
       uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
       if (!B_ROW) {
-        load_block_scales(p, nb, 0, kFp32, cur0, cur1);
-        load_block_scales(p, nb, 32, kFp32, nxt0, nxt1);
+        // lane l holds K block (kb0 rounded down to 32) + l, then the next 32
+        const int base = u.kb0 & ~31;
+        load_block_scales(p, nb, base, kFp32, cur0, cur1);
+        load_block_scales(p, nb, base + 32, kFp32, nxt0, nxt1);
       }
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
         const int s = it % P_STAGES;
         const uint32_t ph = (it / P_STAGES) & 1;
-        if (!B_ROW && kb > 0 && (kb & 31) == 0) {
+        if (!B_ROW && kb > u.kb0 && (kb & 31) == 0) {
           cur0 = nxt0;
           cur1 = nxt1;
           load_block_scales(p, nb, kb + 32, kFp32, nxt0, nxt1);
@@ -896,16 +979,16 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     const int row_in_tile = 32 * quarter + lane;
     uint8_t* stage = smem + C::kOffStage + ew * C::kStage;
     const uint32_t tempty_leader0 = mapa_shared(tempty_bar(0), 0);
-    uint32_t it = 0, tcount = 0;
+    uint32_t it = 0, tcount = 0, nload = 0;
     bool ok = true;
-    for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
+    for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
       float2 acc[kAcc];
       if (kFp32) {
 #pragma unroll
         for (int i = 0; i < kAcc; ++i) acc[i] = make_float2(0.0f, 0.0f);
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
           const uint32_t b = it & 1;
@@ -964,10 +1047,84 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
-      if constexpr (ACC)
-        add_boxes_f32<kCols / 32>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
-      else
+      if constexpr (ACC) {
+        add_boxes_f32<kCols / 32>(&p.tmD, p.N, p.M, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+      } else {
+        if (u.split) {
+          const int sub = 8 * static_cast<int>(rank) + ew;  // this warp's slice of the tile
+          const int wrow = P_BMC * static_cast<int>(rank) + 32 * quarter;
+          // In the cluster's last unit the operand stages are idle once its
+          // accumulator is complete: each epilogue warp then stages its whole
+          // 32 x 128 FP32 slice (four 32 x 32 boxes) in 16 KB of them.
+          const bool last = next_unit(p, u, cl, ncl).tile < 0;
+          const uint32_t big = smem_u32(smem + C::kOffA + ew * 16384);
+          if (u.kb0 > 0) {
+            // not the head piece: partial sum into this cluster's slot, then
+            // the flag (release, after the stores have been performed)
+            if (last) {
+#pragma unroll
+              for (int j = 0; j < kCols / 32; ++j)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                  const int q = 16 * j + 2 * c;
+                  st_shared_v4f(big + 4096 * j + 128 * lane + 16 * (c ^ (lane & 7)), acc[q].x, acc[q].y, acc[q + 1].x,
+                                acc[q + 1].y);
+                }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                for (int j = 0; j < kCols / 32; ++j)
+                  tma_store_2d(&p.tmW, big + 4096 * j, slice * kCols + 32 * j, cl * 256 + wrow);
+                bulk_commit_group();
+              }
+            } else {
+              store_boxes_f32<kCols / 32>(&p.tmW, acc, stage, lane, cl * 256 + wrow, slice * kCols);
+            }
+            if (lane == 0) {
+              bulk_wait_group0();
+              fence_proxy_async_global();
+              st_release_gpu(p.ws_flag + 16 * cl + sub, 1);
+            }
+            __syncwarp();
+            continue;
+          }
+          // head piece (always its cluster's last unit): add the partials of
+          // the clusters whose ranges start inside this tile, in cluster
+          // order, each brought in by four TMA box loads; reset their flags
+          const int64_t tile_end = static_cast<int64_t>(u.tile - p.dp_tiles + 1) * p.num_kb;
+          for (int c = cl + 1; c < ncl && split_bound(p, c, ncl) < tile_end; ++c) {
+            int* flag = p.ws_flag + 16 * c + sub;
+            bool got = true;
+            if (lane == 0) {
+              got = flag_wait(flag, 1, guard, kTimeoutSplit);
+              if (got) {
+                fence_proxy_async_global();
+                mbar_arrive_expect_tx(eload_bar(ew), 4096u * (kCols / 32));
+                for (int j = 0; j < kCols / 32; ++j)
+                  tma_load_2d(big + 4096 * j, &p.tmW, eload_bar(ew), slice * kCols + 32 * j, c * 256 + wrow);
+              }
+            }
+            if (!__all_sync(0xffffffffu, __shfl_sync(0xffffffffu, got, 0))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(eload_bar(ew), nload & 1, guard, kTimeoutSplit))) { ok = false; break; }
+            ++nload;
+#pragma unroll
+            for (int j = 0; j < kCols / 32; ++j)
+#pragma unroll
+              for (int cc = 0; cc < 8; ++cc) {
+                const int q = 16 * j + 2 * cc;
+                const float4 v = ld_shared_v4f(big + 4096 * j + 128 * lane + 16 * (cc ^ (lane & 7)));
+                acc[q] = __fadd2_rn(acc[q], make_float2(v.x, v.y));
+                acc[q + 1] = __fadd2_rn(acc[q + 1], make_float2(v.z, v.w));
+              }
+            fence_proxy_async_smem();  // these reads before the next loads into the buffer
+            __syncwarp();
+            if (lane == 0) *flag = 0;
+          }
+          if (!ok) break;
+          (void)last;
+        }
         store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+      }
     }
     if (lane == 0) bulk_wait_group0();
     __syncwarp();
@@ -1464,8 +1621,39 @@ bool encode_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
   return r == CUDA_SUCCESS;
 }
 
+// Whole tiles take ceil(T / C) rounds on C clusters, the last one R / C full
+// (R = T mod C).  With a workspace, the R tiles of that round are split along
+// K over all C clusters (about W + R / C rounds, W = T / C) when there is at
+// least one full round, the split saves more than 5% of the launch, each
+// cluster gets at least four K blocks and the workspace has a slot per
+// cluster.  Not for FP32 accumulation.  (With fewer tiles than clusters,
+// measured on the layer's O-projection weight gradient, every tile splits
+// into two pieces and the launch got slower, not faster: the SM clock the
+// tensor cores sustain drops as more of them run, which takes back most of
+// what the idle clusters would have added.)
+bool split_tiles(Params& prm, int C, const GemmProblem& pr) {
+  const int T = prm.num_tiles, W = T / C, R = T % C;
+  const int64_t slots = pr.ws != nullptr ? pr.ws_bytes / kWsSlotBytes : 0;
+  if (pr.acc_f32 || W == 0 || R == 0 || slots < C) return false;
+  if (20LL * (C - R) <= static_cast<int64_t>(C) * (W + 1)) return false;
+  if (static_cast<int64_t>(R) * prm.num_kb < 4LL * C) return false;
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {256, static_cast<cuuint64_t>(slots) * 256};
+  cuuint64_t strides[1] = {256 * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t es[2] = {1, 1};
+  if (fn(&prm.tmW, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, pr.ws, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  prm.ws = static_cast<float*>(pr.ws);
+  prm.ws_flag = reinterpret_cast<int*>(static_cast<uint8_t*>(pr.ws) + slots * kWsTileBytes);
+  prm.dp_tiles = W * C;
+  return true;
+}
+
 template <int FMT, bool BK_, bool BR_, bool ACC_ = false>
-cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cudaStream_t stream) {
+cudaError_t launch_pair_variant(Params& prm, const GemmProblem& pr, DeviceInfo* di, int slot, cudaStream_t stream) {
   auto kern = gemm_pair_kernel<FMT, BK_, BR_, ACC_>;
   constexpr uint32_t kSmem = pairk::Cfg<FMT == kFmtFp32>::kSmemAlloc;
   if (!di->pair_attr_set[slot]) {
@@ -1489,7 +1677,8 @@ cudaError_t launch_pair_variant(const Params& prm, DeviceInfo* di, int slot, cud
     di->pair_clusters[slot] = ncl;
     di->pair_attr_set[slot] = true;
   }
-  const int ncl = prm.num_tiles < di->pair_clusters[slot] ? prm.num_tiles : di->pair_clusters[slot];
+  int ncl = prm.num_tiles < di->pair_clusters[slot] ? prm.num_tiles : di->pair_clusters[slot];
+  if (split_tiles(prm, di->pair_clusters[slot], pr)) ncl = di->pair_clusters[slot];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ncl, 1, 1);
   cfg.blockDim = dim3(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1, 1);
@@ -1658,6 +1847,7 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.num_n = static_cast<int>((pr.N + BN - 1) / BN);
   prm.num_tiles = prm.num_m * prm.num_n;
   prm.num_kb = static_cast<int>(pr.K / BK);
+  prm.dp_tiles = prm.num_tiles;  // nothing split unless the pair launcher splits
   prm.status = di->status;
   prm.limit_ns = 2000000000ull;  // 2 s per wait
   const int grid = prm.num_tiles < di->sms ? prm.num_tiles : di->sms;
@@ -1676,20 +1866,20 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
     return launch_fused_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
   }
   if (acc) {
-    if (mx) return launch_pair_variant<kFmtMx, true, true, true>(prm, di, 9, stream);
-    if (fp32) return launch_pair_variant<kFmtFp32, true, true, true>(prm, di, 7, stream);
-    return launch_pair_variant<kFmtUe8m0, true, true, true>(prm, di, 8, stream);
+    if (mx) return launch_pair_variant<kFmtMx, true, true, true>(prm, pr, di, 9, stream);
+    if (fp32) return launch_pair_variant<kFmtFp32, true, true, true>(prm, pr, di, 7, stream);
+    return launch_pair_variant<kFmtUe8m0, true, true, true>(prm, pr, di, 8, stream);
   }
-  if (mx) return launch_pair_variant<kFmtMx, true, true>(prm, di, 6, stream);
+  if (mx) return launch_pair_variant<kFmtMx, true, true>(prm, pr, di, 6, stream);
   if (pair) {
     if (fp32) {
-      if (bk && !br) return launch_pair_variant<kFmtFp32, true, false>(prm, di, 0, stream);
-      if (!bk && !br) return launch_pair_variant<kFmtFp32, false, false>(prm, di, 1, stream);
-      return launch_pair_variant<kFmtFp32, true, true>(prm, di, 2, stream);
+      if (bk && !br) return launch_pair_variant<kFmtFp32, true, false>(prm, pr, di, 0, stream);
+      if (!bk && !br) return launch_pair_variant<kFmtFp32, false, false>(prm, pr, di, 1, stream);
+      return launch_pair_variant<kFmtFp32, true, true>(prm, pr, di, 2, stream);
     }
-    if (bk && !br) return launch_pair_variant<kFmtUe8m0, true, false>(prm, di, 3, stream);
-    if (!bk && !br) return launch_pair_variant<kFmtUe8m0, false, false>(prm, di, 4, stream);
-    return launch_pair_variant<kFmtUe8m0, true, true>(prm, di, 5, stream);
+    if (bk && !br) return launch_pair_variant<kFmtUe8m0, true, false>(prm, pr, di, 3, stream);
+    if (!bk && !br) return launch_pair_variant<kFmtUe8m0, false, false>(prm, pr, di, 4, stream);
+    return launch_pair_variant<kFmtUe8m0, true, true>(prm, pr, di, 5, stream);
   }
   if (fp32) {
     if (bk && !br) return launch_variant<kFmtFp32, true, false>(prm, grid, di, 0, stream);

@@ -49,7 +49,14 @@ struct GemmProblem {
   int64_t M, N, K, ldd;
   int fmt;        // kFmtFp32 / kFmtUe8m0 (both operands)
   bool acc_f32;   // D is FP32 and accumulated into (D += A B^T); else BF16 D = A B^T
+  void* ws = nullptr;    // split-tile workspace (flags zero between calls), or none
+  int64_t ws_bytes = 0;
 };
+
+// Split-tile workspace: one slot of a 256 x 256 FP32 partial sum per CTA
+// pair, then 16 int flags per slot (one per epilogue warp slice of the pair).
+constexpr int64_t kWsTileBytes = 256 * 256 * 4;
+constexpr int64_t kWsSlotBytes = kWsTileBytes + 16 * 4;
 
 // Launches the GEMM; returns a cudaError_t (cudaSuccess on success).  Sets
 // *unsupported when the operand combination is not built.

@@ -78,6 +78,33 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   return mbar_wait_slow(bar, parity, g, code);
 }
 
+// ------------------------------------------------- flags in global memory --
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Bounded wait for *flag == want (acquire), with the mbarrier waits' timeout
+// and abort rules.
+static __device__ __noinline__ bool flag_wait(const int* flag, int want, const WaitGuard& g, int code) {
+  const uint64_t start = global_timer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (ld_acquire_gpu(flag) == want) return true;
+    if ((i & 15u) == 15u) {
+      if (*g.abort_flag) return false;
+      if (global_timer_ns() - start > g.limit_ns) {
+        *g.abort_flag = 1;
+        atomicCAS(g.status, 0, code);
+        return false;
+      }
+    }
+    __nanosleep(100);
+  }
+}
+
 // ------------------------------------------------------------------ TMA --
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int32_t c0, int32_t c1) {
@@ -111,6 +138,11 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 // proxy (TMA, tcgen05.cp, tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's async-proxy accesses of global memory (bulk copies,
+// reduce-adds) with its later generic-proxy accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // -------------------------------------------------------------- tcgen05 --
@@ -440,6 +472,11 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 // move into integer registers first).
 __device__ __forceinline__ void st_shared_v4f(uint32_t addr, float a, float b, float c, float d) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d));
+}
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
 }
 __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   uint32_t v;

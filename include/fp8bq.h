@@ -237,6 +237,44 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream);
 
+/*
+ * fp8bq_gemm with a workspace that lets the kernel split tiles along K
+ * (same product, same arguments and errors as fp8bq_gemm; the pages have no
+ * counterpart: it is how the GEMM above fills a B200).  On C CTA pairs
+ * (C = multiprocessors / 2) T output tiles of 256 x 256 take ceil(T / C)
+ * rounds, the last one (T mod C) / C full; for the weight-gradient shapes of
+ * the layer that round is mostly idle.  With a workspace, the tiles of that
+ * round are shared along K by all C pairs, each pair taking one contiguous
+ * run of their K blocks.  A tile's head piece (from K block 0) adds the FP32
+ * partial sums that the tile's other pieces stored in their pairs' workspace
+ * slots, in pair order, and rounds the tile to BF16 once: results are
+ * bitwise reproducible, though not bitwise equal to fp8bq_gemm's (the same
+ * FP32 sums, grouped differently).  The kernel splits only when there are
+ * more tiles than CTA pairs and the split saves more than 5% of the launch.
+ * Not used with FP8BQ_GEMM_ACCUMULATE_F32 (the workspace is then ignored).
+ * The pieces of a tile wait for one another, so a split launch needs all its
+ * CTA pairs resident at once (the GPU's SMs not held by other work); when
+ * they cannot be, the waits expire after 2 s and fp8bq_check() reports
+ * ERR_TIMEOUT.  Nothing is split when fewer than 4 K blocks per pair result.
+ *   workspace        device memory of workspace_bytes, 256-byte aligned, all
+ *                    zero before its first use; every call that completes
+ *                    leaves its flags zero again.  After a call that fails on
+ *                    the device (ERR_TIMEOUT), zero it before the next use.
+ *                    Calls that may run at the same time need workspaces of
+ *                    their own.  NULL: as fp8bq_gemm.
+ *   workspace_bytes  at least fp8bq_gemm_workspace_bytes() (one 256 KB + 64
+ *                    byte slot per CTA pair); a smaller workspace splits
+ *                    nothing.
+ * Errors: as fp8bq_gemm; ERR_INVALID_ARG for workspace_bytes < 0, ERR_ALIGN
+ * for a workspace not 256-byte aligned.
+ */
+int fp8bq_gemm_ws(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
+                  int64_t ldd, uint32_t flags, void* workspace, int64_t workspace_bytes, fp8bq_stream_t stream);
+
+/* Workspace bytes for fp8bq_gemm_ws on the current device (one slot per CTA
+ * pair), or -1 when no usable device is current. */
+int64_t fp8bq_gemm_workspace_bytes(void);
+
 /* Row stride of a 1x128-group scale array: rows rounded up to 128. */
 int64_t fp8bq_row_scale_ld(int64_t rows);
 

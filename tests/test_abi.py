@@ -166,3 +166,14 @@ def test_gemm_argument_checks(L):
     assert g(A, _op(L, k_major=0, ld=256)) == UNSUPPORTED   # row-group B must be k-major
     assert g(A, _op(L, gran=1, s_stride_k=3, s_stride_r=3)) == SHAPE  # neither layout
     assert g(A, _op(L, dtype=1, scales=0, ld=512)) == UNSUPPORTED      # BF16 B
+
+
+def test_gemm_ws_argument_checks(L):
+    f = L.fp8bq_gemm_ws
+    A = _op(L)
+    B = _op(L, gran=1, s_stride_k=2, s_stride_r=1)
+    g = lambda ws, nbytes: f(ctypes.byref(A), ctypes.byref(B), P, 256, 256, 512, 256, 0, ws, nbytes, None)
+    assert g(P + 16, 1 << 24) == ALIGN        # workspace must be 256-byte aligned
+    assert g(P, -1) == INVALID
+    assert g(None, 0) in (CUDA, UNSUPPORTED)  # no workspace: fp8bq_gemm, which then finds no device
+    assert L.fp8bq_gemm_workspace_bytes() == -1  # no usable device here
