@@ -275,6 +275,30 @@ int fp8bq_gemm_ws(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64
  * pair), or -1 when no usable device is current. */
 int64_t fp8bq_gemm_workspace_bytes(void);
 
+/*
+ * fp8bq_gemm_ws for callers that cannot allocate device memory: the
+ * workspace is a fixed array inside this library instead of memory the
+ * caller provides.  The pages have no counterpart; it exists for callers
+ * that may not call cudaMalloc (it can synchronize the device, stalling
+ * other streams), whose device memory is already held by another allocator,
+ * or that are handed only their inputs and outputs, as plugin interfaces do.
+ * Same arguments, product and errors as fp8bq_gemm, and the same tiles
+ * split as fp8bq_gemm_ws with a workspace of fp8bq_gemm_workspace_bytes().
+ *   Limit: the array has slots for 80 CTA pairs (20.98 MB, held on every GPU
+ *   that loads the library until the process exits); on a device with more
+ *   than 160 multiprocessors the call returns ERR_UNSUPPORTED.  Nothing is
+ *   allocated: no cudaMalloc, no cudaFree.
+ *   The first call on each device looks up the array's device address with
+ *   that device current (cudaGetSymbolAddress); make that first call before
+ *   any stream capture.  Every call then clears the array's flag words on
+ *   the stream (cudaMemsetAsync) before the GEMM.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents: calls that may overlap on the GPU (other streams, other host
+ *   threads) race on it and must be ordered by the caller.
+ */
+int fp8bq_gemm_noalloc(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
+                       int64_t ldd, uint32_t flags, fp8bq_stream_t stream);
+
 /* Row stride of a 1x128-group scale array: rows rounded up to 128. */
 int64_t fp8bq_row_scale_ld(int64_t rows);
 

@@ -177,3 +177,12 @@ def test_gemm_ws_argument_checks(L):
     assert g(P, -1) == INVALID
     assert g(None, 0) in (CUDA, UNSUPPORTED)  # no workspace: fp8bq_gemm, which then finds no device
     assert L.fp8bq_gemm_workspace_bytes() == -1  # no usable device here
+
+
+def test_gemm_noalloc_argument_checks(L):
+    f = L.fp8bq_gemm_noalloc
+    A = _op(L)
+    B = _op(L, gran=1, s_stride_k=2, s_stride_r=1)
+    assert f(None, ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == INVALID
+    assert f(ctypes.byref(A), ctypes.byref(B), None, 256, 256, 512, 256, 0, None) == INVALID
+    assert f(ctypes.byref(A), ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == UNSUPPORTED  # no device here
