@@ -573,6 +573,15 @@ def case_launchers(step, fp):
             it["gu"] = torch.randn(M, 2 * K, generator=gen, device=it["x"].device).to(torch.bfloat16)
             out[f"quant_swiglu:{n}"] = ("quant", M * 2 * K * 2 + 2 * M * K + 2 * (K // 128) * M * sb,
                                         lambda it=it: fp.swiglu_quantize(it["gu"], f))
+        if n in ("qkv", "gate_up"):
+            # the projection's input from RMSNorm in one pass: rstd, h = x * rstd * gamma,
+            # both code layouts (vs a BF16 h written and read back)
+            it["gamma"] = (1.0 + 0.1 * torch.randn(K, device=it["x"].device)).to(torch.bfloat16)
+            it["rstd"] = torch.empty(M, dtype=torch.float32, device=it["x"].device)
+            out[f"quant_rmsnorm:{n}"] = ("quant", M * K * 4 + ((K // 128) * M + (M // 128) * K) * sb + 4 * M + 2 * K,
+                                         lambda it=it: fp.rmsnorm_quantize(
+                                             it["x"], it["gamma"], 1e-6, f,
+                                             out=(it["qx"], it["sx"], it["qxt"], it["sxt"], None, it["rstd"])))
         # fused quantize-on-load: BF16 A quantized inside the GEMM
         out[f"gemm_fwd_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=step.ws))

@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
     "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
-    "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "Operand",
+    "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "rmsnorm_quantize",
+    "Operand",
     "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "gemm_workspace", "linear_forward",
     "linear_dgrad", "linear_wgrad", "check",
 ]
@@ -85,6 +86,8 @@ def lib():
             getattr(L, name).argtypes = [vp, i64, i64, i64, vp, vp, vp]
         L.fp8bq_swiglu_quantize.restype = i32
         L.fp8bq_swiglu_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
+        L.fp8bq_rmsnorm_quantize.restype = i32
+        L.fp8bq_rmsnorm_quantize.argtypes = [vp, i64, i64, i64, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, vp]
         L.fp8bq_quantize_act_dual_mx.restype = i32
         L.fp8bq_quantize_act_dual_mx.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.fp8bq_gemm.restype = i32
@@ -212,6 +215,32 @@ def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = 
                                      ptr(qt), ptr(st), fmt, _stream(gu))
     _raise(rc, "fp8bq_swiglu_quantize")
     return q, s, qt, st, h
+
+
+def rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, fmt: int = SCALE_FP32,
+                     transposed: bool = True, keep_h: bool = False, out=None):
+    """x bf16 [M, K], gamma bf16 [K] -> (q, s, qt, st, h, rstd): h = x * rstd * gamma in
+    BF16 (rstd = 1 / sqrt(mean(x^2) + eps), fp32 [M]) quantized as quantize_act (q, s)
+    and, with transposed, quantize_act_t (qt, st); h is returned when keep_h (else
+    None), qt/st are None without transposed.  `out` may pass (q, s, qt, st, h, rstd)
+    to write into."""
+    _check_bf16(x, "x")
+    M, K = x.shape
+    if (not gamma.is_cuda or gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_contiguous()
+            or gamma.device != x.device):
+        raise ValueError("gamma must be a contiguous bf16 CUDA tensor of K entries on x's device")
+    o = list(out) if out is not None else [None] * 6
+    q = _out(o[0], (M, K), torch.float8_e4m3fn, x.device)
+    s = _out(o[1], (K // 128, row_scale_ld(M)), _scale_dtype(fmt), x.device)
+    qt = _out(o[2], (K, M), torch.float8_e4m3fn, x.device) if transposed else None
+    st = _out(o[3], (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device) if transposed else None
+    h = _out(o[4], (M, K), torch.bfloat16, x.device) if keep_h else None
+    rstd = _out(o[5], (M,), torch.float32, x.device)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    rc = lib().fp8bq_rmsnorm_quantize(x.data_ptr(), M, K, x.stride(0), gamma.data_ptr(), float(eps), rstd.data_ptr(),
+                                      ptr(h), q.data_ptr(), s.data_ptr(), ptr(qt), ptr(st), fmt, _stream(x))
+    _raise(rc, "fp8bq_rmsnorm_quantize")
+    return q, s, qt, st, h, rstd
 
 
 def quantize_act_mx(x: torch.Tensor, q=None, s=None):

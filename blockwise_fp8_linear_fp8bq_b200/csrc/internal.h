@@ -22,6 +22,9 @@ cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx,
 // (row groups, and token groups when qt != nullptr); h optionally stored.
 cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* s_rows,
                                 void* qt, void* s_cols, int fmt, cudaStream_t stream);
+cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
+                                 float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
+                                 cudaStream_t stream);
 
 // Driver entry point of cuTensorMapEncodeTiled (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();

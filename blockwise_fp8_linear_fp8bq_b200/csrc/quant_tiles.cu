@@ -65,9 +65,20 @@ struct QParams {
   uint64_t limit_ns;
   // SwiGLU producer: X is h = silu(gate) * up of tmX's [gate | up] columns
   int64_t up_off;   // column of up[0] (= F)
-  uint16_t* h;      // optional BF16 h [M, K] (ld ldh) written on the way
+  uint16_t* h;      // optional BF16 h [M, K] (ld ldh) written on the way (SwiGLU or RMSNorm)
   int64_t ldh;
+  // RMSNorm producer: X is h = x * rstd[row] * gamma[col]
+  const float* rstd;       // [M]
+  const uint16_t* gamma;   // BF16 [K]
 };
+
+// h = x * rstd * gamma in fp32 (two roundings), rounded to bf16 (nearest,
+// ties to even): within one bf16 ulp of the exact product.  g is the pair's
+// gamma, already in fp32.
+__device__ __forceinline__ uint32_t rmsnorm_bf16x2(uint32_t x2, float2 rs2, float2 g) {
+  const float2 h = __fmul2_rn(__fmul2_rn(make_float2(bf16_lo(x2), bf16_hi(x2)), rs2), g);
+  return pack_bf16x2(h.x, h.y);
+}
 
 // h = silu(g) u = g u / (1 + e^-g) in fp32, rounded to bf16 (nearest, ties
 // to even; finite values).  The fast exponential and division keep the fp32
@@ -76,17 +87,14 @@ struct QParams {
 // except next to a rounding boundary.  For gate < -87, e^-g overflows and
 // h = +-0.
 __device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
-  uint32_t out = 0;
+  float h[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
     const float g = k ? bf16_hi(g2) : bf16_lo(g2);
     const float u = k ? bf16_hi(u2) : bf16_lo(u2);
-    const float h = __fdividef(g * u, 1.0f + __expf(-g));
-    const uint32_t b = __float_as_uint(h);
-    const uint32_t r = (b + 0x7FFFu + ((b >> 16) & 1u)) >> 16;
-    out |= r << (16 * k);
+    h[k] = __fdividef(g * u, 1.0f + __expf(-g));
   }
-  return out;
+  return pack_bf16x2(h[0], h[1]);  // round to nearest even
 }
 
 // Byte offset of 16-byte chunk c (0..15, 8 bf16 each) of tile row r: chunks
@@ -266,7 +274,7 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   }
 }
 
-template <int FMT, bool ROWS, bool COLS, int G, bool SW>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW, bool NORM>
 __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_constant__ QParams p) {
   static_assert(G == 128 || (G == 32 && FMT == kFmtUe8m0), "1x32 groups use UE8M0 scales");
   using C = QCfg<SW>;
@@ -332,6 +340,22 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       mbar_wait(full_bar(j % S), (j / S) & 1, guard, kQTimeoutProducer);
   } else {
     // ------------------------------------------------------------ consumers
+    // RMSNorm: gamma of this thread's 8 columns and rstd of its 4 rows, for
+    // the tile at hand (loaded one tile ahead, off the critical path)
+    uint4 ng = make_uint4(0, 0, 0, 0);
+    float nrs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    auto norm_load = [&](int tile) {
+      if (tile >= p.num_tiles) return;
+      const int64_t tm0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
+      const int64_t tk0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
+      ng = __ldg(reinterpret_cast<const uint4*>(p.gamma + tk0 + 8 * (threadIdx.x % 16)));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t r = tm0 + threadIdx.x / 16 + 32 * i;
+        nrs[i] = r < p.M ? __ldg(p.rstd + r) : 0.0f;
+      }
+    };
+    if constexpr (NORM) norm_load(blockIdx.x);
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++it) {
       const int s = it % S;
@@ -355,6 +379,31 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
           st_shared_v4(base + off, h.x, h.y, h.z, h.w);
           if (p.h != nullptr && m0 + r < p.M)
             *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + k0 + 8 * (t % 16)) = h;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(hready_bar(s));
+        if (!__all_sync(0xffffffffu, mbar_wait(hready_bar(s), ph, guard, kQTimeoutConsumer))) break;
+      } else if constexpr (NORM) {
+        // h = x * rstd * gamma over the tile, in place: thread t takes chunk
+        // t % 16 (gamma of those 8 columns) of rows t / 16 + 32 i
+        const int t = threadIdx.x;
+        const int64_t col = k0 + 8 * (t % 16);
+        const float2 g0 = make_float2(bf16_lo(ng.x), bf16_hi(ng.x)), g1 = make_float2(bf16_lo(ng.y), bf16_hi(ng.y));
+        const float2 g2 = make_float2(bf16_lo(ng.z), bf16_hi(ng.z)), g3 = make_float2(bf16_lo(ng.w), bf16_hi(ng.w));
+        float rsv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rsv[i] = nrs[i];
+        norm_load(tile + gridDim.x);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = t / 16 + 32 * i;
+          const uint32_t off = tile_chunk(r, t % 16);
+          const float2 rs2 = make_float2(rsv[i], rsv[i]);
+          const uint4 x = ld_shared_v4(base + off);
+          const uint4 h = make_uint4(rmsnorm_bf16x2(x.x, rs2, g0), rmsnorm_bf16x2(x.y, rs2, g1),
+                                     rmsnorm_bf16x2(x.z, rs2, g2), rmsnorm_bf16x2(x.w, rs2, g3));
+          st_shared_v4(base + off, h.x, h.y, h.z, h.w);
+          if (p.h != nullptr && m0 + r < p.M) *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + col) = h;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(hready_bar(s));
@@ -383,9 +432,9 @@ bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64
   return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool ROWS, bool COLS, int G, bool SW = false>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW = false, bool NORM = false>
 cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
-  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G, SW>;
+  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G, SW, NORM>;
   constexpr uint32_t kQSmem = QCfg<SW>::kSmem;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -486,6 +535,80 @@ cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ld
                 : launch_tiles<kFmtFp32, true, false, 128, true>(prm, stream);
   return cols ? launch_tiles<kFmtUe8m0, true, true, 128, true>(prm, stream)
               : launch_tiles<kFmtUe8m0, true, false, 128, true>(prm, stream);
+}
+
+namespace {
+
+// rstd[r] = 1 / sqrt(mean_k x[r, k]^2 + eps) in fp32 (IEEE square root and
+// division): one warp per row, 8 values a lane per step, tree reduction.
+__global__ void __launch_bounds__(256) rstd_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx,
+                                                   float eps, float* __restrict__ rstd) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= M) return;
+  const uint16_t* row = x + r * ldx;
+  float acc = 0.0f;
+#pragma unroll 4
+  for (int64_t k = 8 * lane; k < K; k += 256) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(row + k));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = bf16_lo(w[i]), b = bf16_hi(w[i]);
+      acc = fmaf(a, a, acc);
+      acc = fmaf(b, b, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) rstd[r] = __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(acc, static_cast<float>(K)) + eps));
+}
+
+}  // namespace
+
+// RMSNorm fused with the quantization of its output: x BF16 [M, K] ->
+// rstd [M] (fp32) -> h = x * rstd * gamma (BF16, optionally stored to h
+// [M, K]), quantized as quantize_act (q, s_rows) and, when qt != nullptr, as
+// quantize_act_t (qt, s_cols).  K % 128 == 0; M % 128 == 0 when qt is set.
+cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
+                                 float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
+                                 cudaStream_t stream) {
+  const int64_t blocks = (M + 7) / 8;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  rstd_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), M, K, ldx, eps,
+                                                                 rstd);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  QParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  if (!encode_x(&prm.tmX, x, M, K, ldx)) return cudaErrorInvalidValue;
+  prm.M = M;
+  prm.K = K;
+  prm.q = static_cast<uint8_t*>(q);
+  prm.s_rows = s_rows;
+  prm.lds_m = round_up128(M);
+  prm.qt = static_cast<uint8_t*>(qt);
+  prm.s_cols = s_cols;
+  prm.lds_k = round_up128(K);
+  prm.tiles_k = static_cast<int>(K / 128);
+  const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
+  if (tiles > INT32_MAX) return cudaErrorInvalidValue;
+  prm.num_tiles = static_cast<int>(tiles);
+  prm.h = static_cast<uint16_t*>(h);
+  prm.ldh = K;
+  prm.rstd = rstd;
+  prm.gamma = static_cast<const uint16_t*>(gamma);
+  int* status = nullptr;
+  e = device_status_word(&status);
+  if (e != cudaSuccess) return e;
+  prm.status = status;
+  prm.limit_ns = 2000000000ull;
+  const bool cols = qt != nullptr;
+  if (fmt == kFmtFp32)
+    return cols ? launch_tiles<kFmtFp32, true, true, 128, false, true>(prm, stream)
+                : launch_tiles<kFmtFp32, true, false, 128, false, true>(prm, stream);
+  return cols ? launch_tiles<kFmtUe8m0, true, true, 128, false, true>(prm, stream)
+              : launch_tiles<kFmtUe8m0, true, false, 128, false, true>(prm, stream);
 }
 
 }  // namespace fp8bq

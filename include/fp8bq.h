@@ -174,6 +174,37 @@ int fp8bq_swiglu_quantize(const void* gu, int64_t M, int64_t F, int64_t ldgu, vo
                           void* qt, void* scales_t, int fmt, fp8bq_stream_t stream);
 
 /*
+ * RMSNorm fused with the quantization of its output: the QKV and gate/up
+ * projections' input produced and quantized without a BF16 round trip
+ * through HBM.  The pages keep normalization outside the FP8 matmuls, in
+ * BF16/FP32 ("清华开源 Puro-2B", section "精度"; the digest's "方法": a
+ * Qwen3-1.7B-like model, whose blocks normalize with RMSNorm before these
+ * projections); this call computes that BF16 output and quantizes it.
+ *   x         BF16 [M, K], leading dimension ldx.
+ *   gamma     BF16 [K], the norm's weight (16-byte aligned).
+ *   eps       added to the mean square (finite, >= 0; Qwen3 uses 1e-6).
+ *   rstd      FP32 [M], written: 1 / sqrt(mean_k x[r,k]^2 + eps), IEEE square
+ *             root and division of the FP32 mean square (the value the norm's
+ *             backward pass needs).
+ *   h         optional BF16 [M, K] (ld K): h = x * rstd * gamma in FP32,
+ *             rounded to BF16 (nearest, ties to even); may be NULL.  Within
+ *             one BF16 ulp of the exact value.
+ *   q, scales h quantized as fp8bq_quantize_act of exactly that BF16 h:
+ *             E4M3 [M, K] (ld K), scales [K/128][fp8bq_row_scale_ld(M)].
+ *   qt, scales_t  optional (both or neither): h quantized as
+ *             fp8bq_quantize_act_t: [K, M] (ld M), [M/128][fp8bq_row_scale_ld(K)].
+ *   fmt       FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0.
+ * Two launches on the stream: the row statistics, then the quantizer.
+ * Errors: ERR_INVALID_ARG (null x, gamma, rstd, q or scales; only one of qt,
+ * scales_t; bad fmt or eps), ERR_SHAPE (K % 128 != 0; M % 128 != 0 with qt),
+ * ERR_ALIGN (as fp8bq_quantize_act; gamma, h, qt, scales_t 16-B aligned;
+ * rstd 4-B aligned).
+ */
+int fp8bq_rmsnorm_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
+                           float* rstd, void* h, void* q, void* scales, void* qt, void* scales_t, int fmt,
+                           fp8bq_stream_t stream);
+
+/*
  * MX-block quantization (1x32 groups, UE8M0 scales): the other reading of
  * "MXFP8 on Blackwell" ("方法"), with the OCP Microscaling format's 32-value
  * blocks in place of the 1x128 groups.  Same definitions as the calls above

@@ -21,6 +21,7 @@ from .oracle import (  # noqa: F401
     quantize_act,
     gemm_accumulate,
     swiglu,
+    rmsnorm,
     quantize_act_t,
     quantize_weight,
     row_scale_ld,

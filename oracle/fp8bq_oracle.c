@@ -313,6 +313,32 @@ void oracle_swiglu(const uint16_t* gu, int64_t M, int64_t F, int64_t ld, uint16_
   }
 }
 
+/* The QKV and gate/up projections' input: RMSNorm of the block's input.
+ * x is BF16 [M, K] (ld), gamma BF16 [K]; per row r the mean square
+ * ms = sum_k x[r][k]^2 / K and rstd[r] = 1 / sqrt(ms + eps), then
+ * h[r][k] = x[r][k] * rstd[r] * gamma[k], all in float64 (h64 and rstd64
+ * optional), h rounded once to bfloat16 (ld K): the normalized activation
+ * the layer keeps in BF16 ahead of the FP8 matmuls ("清华开源 Puro-2B",
+ * section "精度"; a Qwen3-like block normalizes before QKV and gate/up). */
+void oracle_rmsnorm(const uint16_t* x, int64_t M, int64_t K, int64_t ld, const uint16_t* gamma, double eps,
+                    uint16_t* h, double* h64, double* rstd64) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < M; r++) {
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; k++) {
+      double v = (double)bf16_to_f32(x[r * ld + k]);
+      ss += v * v;
+    }
+    double rs = 1.0 / sqrt(ss / (double)K + eps);
+    if (rstd64) rstd64[r] = rs;
+    for (int64_t k = 0; k < K; k++) {
+      double v = (double)bf16_to_f32(x[r * ld + k]) * rs * (double)bf16_to_f32(gamma[k]);
+      if (h64) h64[r * K + k] = v;
+      h[r * K + k] = f64_to_bf16_rne(v);
+    }
+  }
+}
+
 /* ------------------------------------------------------------------ GEMM -- */
 
 /* A quantized operand seen as a logical matrix [rows, C] with contraction C:

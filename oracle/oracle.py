@@ -75,6 +75,10 @@ def lib():
         L.oracle_swiglu.restype = None
         L.oracle_swiglu.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                     ctypes.c_void_p, ctypes.c_void_p]
+        L.oracle_rmsnorm.restype = None
+        L.oracle_rmsnorm.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p,
+                                     ctypes.c_void_p]
         _lib = L
     return _lib
 
@@ -89,6 +93,23 @@ def swiglu(gu_bits: np.ndarray, with_f64: bool = False):
     h64 = np.empty((M, F), np.float64) if with_f64 else None
     lib().oracle_swiglu(gu.ctypes.data, M, F, F2, h.ctypes.data, h64.ctypes.data if with_f64 else None)
     return (h, h64) if with_f64 else h
+
+
+def rmsnorm(x_bits: np.ndarray, gamma_bits: np.ndarray, eps: float, with_f64: bool = False):
+    """BF16 bits x [M, K] and gamma [K] -> h BF16 bits [M, K] = RNE_bf16(x * rstd * gamma)
+    with rstd = 1 / sqrt(mean(x^2) + eps), in float64 (and, when with_f64, the float64
+    h and rstd [M] too)."""
+    x = _as_u16(x_bits)
+    g = np.ascontiguousarray(_as_u16(gamma_bits).reshape(-1))
+    M, K = x.shape
+    if g.shape[0] != K:
+        raise ValueError("gamma must have K entries")
+    h = np.empty((M, K), np.uint16)
+    h64 = np.empty((M, K), np.float64) if with_f64 else None
+    rs = np.empty(M, np.float64) if with_f64 else None
+    lib().oracle_rmsnorm(x.ctypes.data, M, K, K, g.ctypes.data, float(eps), h.ctypes.data,
+                         h64.ctypes.data if with_f64 else None, rs.ctypes.data if with_f64 else None)
+    return (h, h64, rs) if with_f64 else h
 
 
 def gemm_accumulate(A: "Operand", B: "Operand", d0: np.ndarray, rows=None, cols=None) -> np.ndarray:
