@@ -211,17 +211,23 @@ class LayerStep:
         CUDA event pair around every launch: ev.append((kind, start, end));
         `external` makes them event-record nodes when captured in a graph."""
         fp, f = self.fp, self.fmt
+        # one event between consecutive launches: the end of launch i is the
+        # start of launch i + 1 (a pair per launch would put two event-record
+        # nodes, and their latency, between every two kernels)
+        prev = [None]
+        if ev is not None:
+            prev[0] = torch.cuda.Event(enable_timing=True, external=external)
+            prev[0].record()
 
         def timed(kind, fn):
             if ev is None:
                 fn()
                 return
-            a = torch.cuda.Event(enable_timing=True, external=external)
-            b = torch.cuda.Event(enable_timing=True, external=external)
-            a.record()
             fn()
+            b = torch.cuda.Event(enable_timing=True, external=external)
             b.record()
-            ev.append((kind, a, b))
+            ev.append((kind, prev[0], b))
+            prev[0] = b
 
         if self.mx:
             for it in self.items:
@@ -281,9 +287,9 @@ def run_ours(args, rank, world, dist):
     # (`value`) holds per step the L2 flush and one event pair around the
     # step: nothing sits between the step's kernels.  The kernel split
     # (`roofline`, `gemm`, `quantizers`) comes from the other graph, replayed
-    # first, which adds an event pair around every launch; those event-record
-    # nodes order the kernels strictly, so its step runs a few percent
-    # longer.  The host's Python and ctypes work is outside both.  (--no-graph
+    # first, which adds an event between every two launches; those
+    # event-record nodes order the kernels strictly, so its step runs a few
+    # percent longer.  The host's Python and ctypes work is outside both.  (--no-graph
     # issues the same two sequences eagerly.)
     step_events, split_step_events, kernel_events = [], [], []
 
@@ -591,6 +597,20 @@ def case_launchers(step, fp):
     return out
 
 
+def lm_head_case(fp, fmt, dev, ws):
+    """The LM head forward GEMM, [16384 x 2048] . [151936 x 2048]^T (10.2 TFLOP):
+    the largest GEMM of the 28-layer sweep, timed as a single kernel."""
+    from blockwise_fp8_linear_fp8bq_b200 import synth
+    lin = synth.LM_HEAD
+    x, w = lin.x(5000, device=dev), lin.w(5000, device=dev)
+    qx, sx = fp.quantize_act(x, fmt)
+    qw, sw = fp.quantize_weight(w, fmt)
+    del x, w
+    y = torch.empty(lin.M, lin.N, dtype=torch.bfloat16, device=dev)
+    A, B = fp.row_operand(qx, sx, fmt), fp.block_operand(qw, sw, fmt)
+    return {"gemm_fwd:lm_head": ("gemm", lin.flops, lambda: fp.gemm(A, B, y, workspace=ws))}
+
+
 def run_case(args):
     """Time single kernels of the step (L2 flushed before every launch).
     --case all prints one line per kernel; --case NAME runs only that kernel
@@ -607,6 +627,8 @@ def run_case(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
     cases = case_launchers(step, fp)
+    if args.scale != "mx" and args.case in ("all", "gemm_fwd:lm_head"):
+        cases.update(lm_head_case(fp, fmt, dev, step.ws))
     names = list(cases) if args.case == "all" else [args.case]
     peaks = measured_peaks()
     rows = []
@@ -742,7 +764,7 @@ def main(argv=None):
                  "launches_per_step": r["gemm_launches"] // args.steps},
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
-        "kernel_split": {"source": "a second replay of the same K steps with an event pair around every launch",
+        "kernel_split": {"source": "a replay, before the timed one, of the same K steps with an event between every two launches",
                          "ms_per_step": split_ms, "clocks": r["clocks_split"]},
     }
     if r["e2e"]:

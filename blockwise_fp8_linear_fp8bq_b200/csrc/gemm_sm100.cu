@@ -1121,7 +1121,6 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             if (lane == 0) *flag = 0;
           }
           if (!ok) break;
-          (void)last;
         }
         store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
       }
