@@ -44,7 +44,7 @@ struct QCfg {
   static constexpr uint32_t kOffBar = kStages * kStage;
   static constexpr uint32_t kNumBars = 3 * kStages;  // full[S], empty[S], hready[S]
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kSmem = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static constexpr uint32_t kSmem = kOffMisc + 16 + 2048;  // + slack for 2048-byte alignment
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -165,30 +165,26 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   }
 }
 
-// Byte i of r moves to byte (i + j) mod 16, for 0 <= j < 8.
-__device__ __forceinline__ uint4 rotate_bytes_up(const uint4& r, int j) {
-  uint32_t x0 = r.x, x1 = r.y, x2 = r.z, x3 = r.w;
-  if (j & 4) {
-    const uint32_t t = x3;
-    x3 = x2;
-    x2 = x1;
-    x1 = x0;
-    x0 = t;
-  }
-  const uint32_t sh = 8u * static_cast<uint32_t>(j & 3);
-  return make_uint4(__funnelshift_l(x3, x0, sh), __funnelshift_l(x0, x1, sh), __funnelshift_l(x1, x2, sh),
-                    __funnelshift_l(x2, x3, sh));
+// Byte i of r moves to byte i ^ j, for 0 <= j < 8: bytes within each word
+// by j & 3 (one byte permute), then words pairwise when j & 4.
+__device__ __forceinline__ uint4 xor_bytes(const uint4& r, int j) {
+  const uint32_t sel = 0x3210u ^ (static_cast<uint32_t>(j & 3) * 0x1111u);
+  const uint32_t x0 = __byte_perm(r.x, 0, sel), x1 = __byte_perm(r.y, 0, sel);
+  const uint32_t x2 = __byte_perm(r.z, 0, sel), x3 = __byte_perm(r.w, 0, sel);
+  return (j & 4) ? make_uint4(x1, x0, x3, x2) : make_uint4(x0, x1, x2, x3);
 }
 
 // Token groups: warp w takes box w & 1 and its column pairs 4 (w >> 1) ..
 // + 3; lane (a = lane >> 3, j = lane & 7) owns pair a (two columns, one
 // 32-bit word per token) and tokens 16 j .. 16 j + 15, so a column's 128
 // tokens sit in the eight lanes of its pair and the amax is a shuffle
-// reduction.  Lane j visits its tokens starting at 16 j + j: the eight lanes
-// of a pair then read eight different swizzle phases and the warp's 32 reads
-// hit 32 banks.  The codes come out in that rotated order and are rotated
-// back before each lane stores its 16 consecutive tokens (8 lanes: one
-// 128-byte row segment of the transposed codes).
+// reduction.  Load i of lane j reads token 16 j + (i ^ j): the eight lanes of
+// a pair then read eight different swizzle phases and the warp's 32 reads
+// hit 32 banks, and with the stage 2048-byte aligned every address is the
+// lane's base XOR a constant.  The codes come out in that order and are
+// permuted back (byte i to byte i ^ j) before each lane stores its 16
+// consecutive tokens (8 lanes: one 128-byte row segment of the transposed
+// codes).
 template <int FMT, int G>
 __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
                                           int lane) {
@@ -196,13 +192,14 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   const int a = lane >> 3;
   const int j = lane & 7;
   const int chunk = warp >> 1;  // 16-byte chunk holding the warp's 4 pairs
-  const uint32_t cbase = base + box * kQBox + 4 * a;
-  uint32_t w[16];  // w[i]: token 16 j + ((i + j) & 15)
+  // token r = 16 j + (i ^ j) sits at cbase + 128 r + 16 (chunk ^ (r & 7));
+  // bits 4-10 of cbase + 2048 j are zero, so that is lbase ^ (128 i + 16 (i & 7))
+  const uint32_t jj = static_cast<uint32_t>(j);
+  const uint32_t lbase = (base + box * kQBox + 4 * a + 2048u * jj) ^ ((jj << 7) | (jj << 4)) ^
+                         (static_cast<uint32_t>(chunk) << 4);
+  uint32_t w[16];  // w[i]: token 16 j + (i ^ j)
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int r = 16 * j + ((i + j) & 15);
-    w[i] = ld_shared_u32(cbase + r * 128 + ((chunk ^ (r & 7)) << 4));
-  }
+  for (int i = 0; i < 16; ++i) w[i] = ld_shared_u32(lbase ^ static_cast<uint32_t>((i << 7) | ((i & 7) << 4)));
   // packed |max| over the 16 tokens (both columns at once), then over the
   // 8 lanes of the pair
   uint32_t m2 = 0;
@@ -253,8 +250,8 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
       cb[h] = quant8_exact<FMT>(wb[h], s1);
     }
   }
-  const uint4 va = rotate_bytes_up(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), j);
-  const uint4 vb = rotate_bytes_up(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), j);
+  const uint4 va = xor_bytes(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), j);
+  const uint4 vb = xor_bytes(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), j);
   const int64_t c = k0 + 64 * box + 2 * (4 * chunk + a);
   const int64_t tok = m0 + 16 * j;
   // the first lane of each token group stores its scale: scales [M/G][lds_k]
@@ -280,8 +277,10 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
   using C = QCfg<SW>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // stages 2048-byte aligned: a token-group lane's row addresses then differ
+  // from one another only in bits 4-10 (see tile_cols)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) &
+                                             ~static_cast<uintptr_t>(2047));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
