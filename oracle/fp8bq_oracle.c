@@ -19,7 +19,7 @@
  *     run on the FP8 path (fine-grained block quantization after DeepSeek-V3);
  *     numerically sensitive work and training state stay BF16/FP32.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent:
  *   - FP8 format: OCP E4M3FN (bias 7, max 448, no infinities, S.1111.111 NaN).
  *   - fp32 scale: s = fl32(amax / 448), s = 1 for an all-zero group;
  *     code q = E4M3_RNE_satfinite(fl32(x / s)).
