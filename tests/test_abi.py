@@ -186,3 +186,44 @@ def test_gemm_noalloc_argument_checks(L):
     assert f(None, ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == INVALID
     assert f(ctypes.byref(A), ctypes.byref(B), None, 256, 256, 512, 256, 0, None) == INVALID
     assert f(ctypes.byref(A), ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == UNSUPPORTED  # no device here
+
+
+def test_swiglu_quantize_argument_checks(L):
+    f = L.fp8bq_swiglu_quantize
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    g = lambda gu=P, M=128, F=128, ld=256, h=None, q=P, s=P, qt=None, st=None, fmt=0: f(gu, M, F, ld, h, q, s, qt, st,
+                                                                                      fmt, None)
+    assert g(gu=None) == INVALID
+    assert g(q=None) == INVALID
+    assert g(qt=P) == INVALID                 # qt without scales_t
+    assert g(fmt=3) == INVALID
+    assert g(F=100, ld=200) == SHAPE          # F % 128
+    assert g(ld=128) == SHAPE                 # ldgu < 2F
+    assert g(M=100, qt=P, st=P) == SHAPE      # tokens % 128 with transposed codes
+    assert g(h=P + 8) == ALIGN
+    assert g(qt=P + 4, st=P) == ALIGN
+    assert g(M=0) == OK                       # empty: no launch
+
+
+def test_rmsnorm_quantize_argument_checks(L):
+    f = L.fp8bq_rmsnorm_quantize
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_void_p]
+    g = lambda x=P, M=128, K=256, ld=256, gamma=P, eps=1e-6, rstd=P, h=None, q=P, s=P, qt=None, st=None, fmt=1: f(
+        x, M, K, ld, gamma, eps, rstd, h, q, s, qt, st, fmt, None)
+    assert g(x=None) == INVALID
+    assert g(gamma=None) == INVALID
+    assert g(rstd=None) == INVALID
+    assert g(eps=-1.0) == INVALID
+    assert g(eps=float("nan")) == INVALID
+    assert g(st=P) == INVALID                 # scales_t without qt
+    assert g(K=200, ld=200) == SHAPE          # K % 128
+    assert g(M=100, qt=P, st=P) == SHAPE      # tokens % 128 with transposed codes
+    assert g(gamma=P + 8) == ALIGN
+    assert g(rstd=P + 2) == ALIGN
+    assert g(x=P + 8) == ALIGN
+    assert g(M=0) == OK                       # empty: no launch
