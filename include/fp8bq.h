@@ -14,7 +14,8 @@
  *
  * Conventions shared by every call:
  *   - All data pointers are DEVICE pointers to caller-owned memory.  The library
- *     allocates no device memory and never frees caller memory.
+ *     allocates no device memory and never frees caller memory (the one array
+ *     it owns, fp8bq_gemm_noalloc's workspace, is part of the loaded library).
  *   - Every compute call is asynchronous on `stream` (NULL = legacy default
  *     stream) and never synchronizes; errors it can see at launch are returned
  *     at once, errors that happen on the device surface at fp8bq_check().
@@ -27,16 +28,17 @@
  *         stride is R rounded up to a multiple of 128 and the pad entries
  *         r >= R hold the neutral scale (1.0f, or the byte 127);
  *       128x128 blocks of W [N,K]: scales[kb * ceil(N/128) + nb];
-       1x32 row groups (MX blocks, the other reading of "MXFP8 on
-         Blackwell": the OCP Microscaling format's 32-value blocks with
-         E8M0 scales): as 1x128 row groups with cb = k / 32.
+ *       1x32 row groups (MX blocks, the other reading of "MXFP8 on
+ *         Blackwell": the OCP Microscaling format's 32-value blocks with
+ *         E8M0 scales): as 1x128 row groups with cb = k / 32.
  *     FP32 scales are `float`; UE8M0 scales are one byte e + 127 meaning 2^e.
  *   - Scale definitions:  FP32: s = fl32(amax / 448) (s = 1 for an all-zero
  *     group), code q = E4M3_RNE_satfinite(fl32(x / s)).  UE8M0: e = the least
  *     integer with amax <= 448 * 2^e, clamped to [-127, 127] (e = 0 for an
  *     all-zero group), q = E4M3_RNE_satfinite(x * 2^-e).
  *   - Return value: FP8BQ_OK or one of the negative FP8BQ_ERR_* codes.  A call
- *     that returns an error has launched nothing.
+ *     that returns an error has launched no kernel and written no caller
+ *     memory (fp8bq_gemm_noalloc may have cleared its own array's flags).
  */
 #ifndef FP8BQ_H
 #define FP8BQ_H
@@ -57,7 +59,7 @@ typedef struct CUstream_st* fp8bq_stream_t;
 #define FP8BQ_ERR_UNSUPPORTED (-4) /* no sm_100 device, or an operand combination   */
                                    /* this library does not build                   */
 #define FP8BQ_ERR_CUDA (-5)        /* a CUDA call failed; see fp8bq_last_cuda_error */
-#define FP8BQ_ERR_TIMEOUT (-6)     /* a bounded wait inside a GEMM kernel expired   */
+#define FP8BQ_ERR_TIMEOUT (-6)     /* a bounded wait inside a kernel expired        */
 
 typedef enum { FP8BQ_SCALE_FP32 = 0, FP8BQ_SCALE_UE8M0 = 1 } fp8bq_scale_fmt;
 typedef enum {
