@@ -39,7 +39,7 @@ def _sources():
 
 def _deps():
     return _sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h"))) + \
-        [os.path.join(INCLUDE, "fp8bq.h")]
+        sorted(glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
 def needs_build() -> bool:

@@ -4,19 +4,53 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "fp8bq.h"
+#include "fp8bq_testing.h"
 #include "internal.h"
+#include "quant_math.cuh"
 
 namespace {
-
 thread_local int t_last_cuda_error = 0;
+}  // namespace
+
+namespace fp8bq {
 
 int cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return FP8BQ_OK;
   t_last_cuda_error = static_cast<int>(e);
   return FP8BQ_ERR_CUDA;
 }
+
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+}  // namespace fp8bq
+
+namespace {
+
+using fp8bq::cuda_status;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -50,14 +84,14 @@ int check_quant_args(const void* x, int64_t rows, int64_t cols, int64_t ld, cons
 }
 
 // Operand checks shared by A and B; fills the internal form.
-int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a, int fmt,
-                    fp8bq::GemmOperand* out) {
+int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a, fp8bq::GemmOperand* out) {
   if (!op || !op->data) return FP8BQ_ERR_INVALID_ARG;
   if (op->dtype != FP8BQ_E4M3 && op->dtype != FP8BQ_BF16) return FP8BQ_ERR_INVALID_ARG;
   if (op->gran != FP8BQ_GRAN_ROW_1x128 && op->gran != FP8BQ_GRAN_BLOCK_128x128 &&
       op->gran != FP8BQ_GRAN_ROW_1x32)
     return FP8BQ_ERR_INVALID_ARG;
-  if (op->fmt != fmt) return FP8BQ_ERR_UNSUPPORTED;
+  if (!valid_fmt(op->fmt)) return FP8BQ_ERR_INVALID_ARG;
+  const int fmt = op->fmt;
   if (op->k_major != 0 && op->k_major != 1) return FP8BQ_ERR_INVALID_ARG;
   const bool bf16 = op->dtype == FP8BQ_BF16;
   if (bf16 && (!is_a || !op->k_major)) return FP8BQ_ERR_UNSUPPORTED;
@@ -97,6 +131,52 @@ int convert_operand(const fp8bq_operand* op, int64_t rows, int64_t K, bool is_a,
 }
 
 }  // namespace
+
+namespace fp8bq {
+
+int validate_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
+                  int64_t ldd, uint32_t flags, GemmProblem* p) {
+  if (!A || !B || !D || !p) return FP8BQ_ERR_INVALID_ARG;
+  if ((flags & ~static_cast<uint32_t>(FP8BQ_GEMM_ACCUMULATE_F32)) != 0) return FP8BQ_ERR_INVALID_ARG;
+  const bool acc = (flags & FP8BQ_GEMM_ACCUMULATE_F32) != 0;
+  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0 || ldd < N) return FP8BQ_ERR_SHAPE;
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BQ_ERR_SHAPE;
+  if (!aligned16(D) || ldd % 8 != 0) return FP8BQ_ERR_ALIGN;
+  int st = convert_operand(A, M, K, true, &p->a);
+  if (st != FP8BQ_OK) return st;
+  st = convert_operand(B, N, K, false, &p->b);
+  if (st != FP8BQ_OK) return st;
+  if (p->a.mx != p->b.mx) return FP8BQ_ERR_UNSUPPORTED;  // MX blocks on both operands or neither
+  // A BF16 A is quantized inside the GEMM in its own format; B must share it
+  if (p->a.bf16 && A->fmt != B->fmt) return FP8BQ_ERR_UNSUPPORTED;
+  // FP32 accumulation is built for the weight-gradient layout only
+  if (acc && (p->a.bf16 || !p->a.row_groups || !p->b.row_groups || !p->b.k_major)) return FP8BQ_ERR_UNSUPPORTED;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  p->d = D;
+  p->M = M;
+  p->N = N;
+  p->K = K;
+  p->ldd = ldd;
+  // both UE8M0: the block-scaled MMA; otherwise the FP32 promotion path, with
+  // an operand's UE8M0 scales decoded to 2^e where they are staged
+  const bool both_u8 = A->fmt == FP8BQ_SCALE_UE8M0 && B->fmt == FP8BQ_SCALE_UE8M0;
+  p->fmt = both_u8 ? kFmtUe8m0 : kFmtFp32;
+  p->a_u8 = !both_u8 && A->fmt == FP8BQ_SCALE_UE8M0;
+  p->b_u8 = !both_u8 && B->fmt == FP8BQ_SCALE_UE8M0;
+  p->acc_f32 = acc;
+  p->ws = nullptr;
+  p->ws_bytes = 0;
+  return FP8BQ_OK;
+}
+
+int run_gemm(const GemmProblem& p, cudaStream_t stream) {
+  bool unsupported = false;
+  cudaError_t e = launch_gemm(p, stream, &unsupported);
+  if (unsupported) return FP8BQ_ERR_UNSUPPORTED;
+  return cuda_status(e);
+}
+
+}  // namespace fp8bq
 
 extern "C" {
 
@@ -229,37 +309,30 @@ int64_t fp8bq_gemm_workspace_bytes(void) {
 
 int fp8bq_gemm_ws(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
                   int64_t ldd, uint32_t flags, void* workspace, int64_t workspace_bytes, fp8bq_stream_t stream) {
-  if (!A || !B || !D) return FP8BQ_ERR_INVALID_ARG;
-  if ((flags & ~static_cast<uint32_t>(FP8BQ_GEMM_ACCUMULATE_F32)) != 0) return FP8BQ_ERR_INVALID_ARG;
-  const bool acc = (flags & FP8BQ_GEMM_ACCUMULATE_F32) != 0;
-  if (!valid_fmt(A->fmt)) return FP8BQ_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || K % 128 != 0 || N % 8 != 0 || ldd < N) return FP8BQ_ERR_SHAPE;
-  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return FP8BQ_ERR_SHAPE;
-  if (!aligned16(D) || ldd % 8 != 0) return FP8BQ_ERR_ALIGN;
   if (workspace != nullptr && workspace_bytes < 0) return FP8BQ_ERR_INVALID_ARG;
   if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8BQ_ERR_ALIGN;
   fp8bq::GemmProblem p;
-  int st = convert_operand(A, M, K, true, A->fmt, &p.a);
+  int st = fp8bq::validate_gemm(A, B, D, M, N, K, ldd, flags, &p);
   if (st != FP8BQ_OK) return st;
-  st = convert_operand(B, N, K, false, A->fmt, &p.b);
-  if (st != FP8BQ_OK) return st;
-  if (p.a.mx != p.b.mx) return FP8BQ_ERR_UNSUPPORTED;  // MX blocks on both operands or neither
-  // FP32 accumulation is built for the weight-gradient layout only
-  if (acc && (p.a.bf16 || !p.a.row_groups || !p.b.row_groups || !p.b.k_major)) return FP8BQ_ERR_UNSUPPORTED;
-  if ((st = device_ok()) != FP8BQ_OK) return st;
-  p.d = D;
-  p.M = M;
-  p.N = N;
-  p.K = K;
-  p.ldd = ldd;
-  p.fmt = A->fmt;
-  p.acc_f32 = acc;
   p.ws = workspace;
   p.ws_bytes = workspace != nullptr ? workspace_bytes : 0;
-  bool unsupported = false;
-  cudaError_t e = fp8bq::launch_gemm(p, reinterpret_cast<cudaStream_t>(stream), &unsupported);
-  if (unsupported) return FP8BQ_ERR_UNSUPPORTED;
-  return cuda_status(e);
+  return fp8bq::run_gemm(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int fp8bq_testing_gemm_ws_withhold(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
+                                   int64_t K, int64_t ldd, uint32_t flags, void* workspace, int64_t workspace_bytes,
+                                   int withhold_pair, int64_t wait_limit_ns, fp8bq_stream_t stream) {
+  if (workspace == nullptr || workspace_bytes < 0 || withhold_pair < 0) return FP8BQ_ERR_INVALID_ARG;
+  if (wait_limit_ns < 100000 || wait_limit_ns > 2000000000LL) return FP8BQ_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8BQ_ERR_ALIGN;
+  fp8bq::GemmProblem p;
+  int st = fp8bq::validate_gemm(A, B, D, M, N, K, ldd, flags, &p);
+  if (st != FP8BQ_OK) return st;
+  p.ws = workspace;
+  p.ws_bytes = workspace_bytes;
+  p.withhold_cluster = withhold_pair;
+  p.wait_limit_ns = static_cast<uint64_t>(wait_limit_ns);
+  return fp8bq::run_gemm(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int64_t fp8bq_row_scale_ld(int64_t rows) { return rows < 0 ? -1 : fp8bq::round_up128(rows); }

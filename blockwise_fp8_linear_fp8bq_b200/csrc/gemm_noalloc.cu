@@ -35,11 +35,16 @@ static __device__ __align__(256) unsigned char g_gemm_scratch[kNoAllocBytes];
 
 namespace {
 
-// Device address of g_gemm_scratch on the current device, looked up once
-// per device (with that device current) and cached; nullptr on failure.
+// Device address of g_gemm_scratch in the context current on this thread.
+// It is looked up (cudaGetSymbolAddress, with the device current) on the
+// first call in each context and cached together with the context's
+// identifier, so a new context on the same device (after cudaDeviceReset, or
+// a context the caller created) is looked up again instead of being handed a
+// stale address.  nullptr on failure, with the CUDA error in *err.
 void* scratch_address(cudaError_t* err) {
   static std::mutex mu;
   static void* addr[64] = {};
+  static unsigned long long ctx[64] = {};
   int dev = 0;
   *err = cudaGetDevice(&dev);
   if (*err != cudaSuccess) return nullptr;
@@ -48,33 +53,41 @@ void* scratch_address(cudaError_t* err) {
     return nullptr;
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
-    void* p = nullptr;
-    *err = cudaGetSymbolAddress(&p, g_gemm_scratch);
-    if (*err != cudaSuccess) return nullptr;
-    addr[dev] = p;
-  }
-  return addr[dev];
+  const unsigned long long id = fp8bq::current_context_id();
+  if (addr[dev] != nullptr && id != 0 && ctx[dev] == id) return addr[dev];
+  void* p = nullptr;
+  *err = cudaGetSymbolAddress(&p, g_gemm_scratch);  // makes the device's context current if none is
+  if (*err != cudaSuccess) return nullptr;
+  addr[dev] = p;
+  ctx[dev] = fp8bq::current_context_id();
+  return p;
 }
 
 }  // namespace
 
 extern "C" int fp8bq_gemm_noalloc(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                                   int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream) {
-  if (!A || !B || !D) return FP8BQ_ERR_INVALID_ARG;
+  // every argument is checked before anything is queued on the stream
+  fp8bq::GemmProblem p;
+  int st = fp8bq::validate_gemm(A, B, D, M, N, K, ldd, flags, &p);
+  if (st != FP8BQ_OK) return st;
   const int64_t need = fp8bq_gemm_workspace_bytes();  // one slot per CTA pair of this device
   if (need < 0) return FP8BQ_ERR_UNSUPPORTED;
   if (need > kNoAllocBytes) return FP8BQ_ERR_UNSUPPORTED;  // more CTA pairs than the array has slots for
-  cudaError_t e = cudaSuccess;
-  void* ws = scratch_address(&e);
-  if (ws == nullptr) return FP8BQ_ERR_CUDA;
-  // The flags after the slots must start at zero; the slots need not (a
-  // piece stores its partial sum before its flag says so).  A completed
-  // call leaves the flags zero, a failed one may not: clear them each time.
-  const int64_t slots = need / fp8bq::kWsSlotBytes;
-  e = cudaMemsetAsync(static_cast<unsigned char*>(ws) + slots * fp8bq::kWsTileBytes, 0,
-                      static_cast<size_t>(slots * (fp8bq::kWsSlotBytes - fp8bq::kWsTileBytes)),
-                      reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return FP8BQ_ERR_CUDA;
-  return fp8bq_gemm_ws(A, B, D, M, N, K, ldd, flags, ws, need, stream);
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!p.acc_f32) {  // FP32 accumulation splits nothing and never touches the array
+    cudaError_t e = cudaSuccess;
+    void* ws = scratch_address(&e);
+    if (ws == nullptr) return fp8bq::cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol);
+    // The flags after the slots must start at zero; the slots need not (a
+    // piece stores its partial sum before its flag says so).  A completed
+    // call leaves the flags zero, a failed one may not: clear them each time.
+    const int64_t slots = need / fp8bq::kWsSlotBytes;
+    e = cudaMemsetAsync(static_cast<unsigned char*>(ws) + slots * fp8bq::kWsTileBytes, 0,
+                        static_cast<size_t>(slots * (fp8bq::kWsSlotBytes - fp8bq::kWsTileBytes)), s);
+    if (e != cudaSuccess) return fp8bq::cuda_status(e);
+    p.ws = ws;
+    p.ws_bytes = need;
+  }
+  return fp8bq::run_gemm(p, s);
 }

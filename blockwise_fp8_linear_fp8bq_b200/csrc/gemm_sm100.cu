@@ -122,7 +122,17 @@ struct Params {
   CUtensorMap tmW;  // workspace [clusters * 256][256] FP32, 32 x 32 boxes, 128-byte swizzle
   float* ws;        // one 256 x 256 partial-sum slot per cluster
   int* ws_flag;     // per slot and epilogue warp slice: 1 = partial stored (0 between calls)
+  // FP32 promotion path with one operand's scales in UE8M0 (a mixed pair):
+  // that operand's scale bytes are staged and decoded to the FP32 value 2^e.
+  int a_u8, b_u8;
+  int withhold_cluster;  // test hook: this pair never raises its split flags (-1: none)
 };
+
+// FP32 value of a UE8M0 scale byte u (2^(u - 127)); u = 0 is the subnormal
+// 2^-127.  The quantizers write u in [0, 254].
+__device__ __forceinline__ uint32_t ue8m0_to_f32_bits(uint32_t u) {
+  return u == 0 ? 0x00400000u : (u << 23);
+}
 
 // ----------------------------------------------------------- work units --
 // A cluster's work: the tiles cl, cl + ncl, ... below dp_tiles, each whole;
@@ -770,15 +780,20 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
       const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
       const int32_t brow = nb * P_BN + P_BNC * static_cast<int>(rank);
-      const uint32_t esz = kFp32 ? 4u : 1u;
+      // scale bytes per entry; a UE8M0 operand of the FP32 path lands as raw
+      // bytes in the slot's staging area and is decoded by the staging warp
+      const uint32_t esz_a = kFp32 && !p.a_u8 ? 4u : 1u;
+      const uint32_t esz_b = kFp32 && !p.b_u8 ? 4u : 1u;
+      const uint32_t dst_a = kFp32 && p.a_u8 ? kSlotTm : kSlotRawA;
+      const uint32_t dst_b = kFp32 && p.b_u8 ? kSlotTm + 128 : kSlotRawB;
       const bool a_sc = row0 < p.sa_stride_k;  // rows past the padded scale rows carry only zeros
       uint32_t b_sc_bytes = 0;
       if (B_ROW) {
         const int64_t left = p.sb_len - static_cast<int64_t>(nb) * P_BN;
-        b_sc_bytes = static_cast<uint32_t>(left < P_BN ? left : P_BN) * esz;
+        b_sc_bytes = static_cast<uint32_t>(left < P_BN ? left : P_BN) * esz_b;
       }
-      const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + row0 * esz;
-      const uint8_t* gb = static_cast<const uint8_t*>(p.sB) + static_cast<int64_t>(nb) * P_BN * esz;
+      const uint8_t* ga = static_cast<const uint8_t*>(p.sA) + row0 * esz_a;
+      const uint8_t* gb = static_cast<const uint8_t*>(p.sB) + static_cast<int64_t>(nb) * P_BN * esz_b;
       for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
         const int s = it % P_STAGES;
         const uint32_t ph = (it / P_STAGES) & 1;
@@ -803,9 +818,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tma_load_2d(smem_u32(slot + kSlotRawA), &p.tmSA, fullsc_bar(s), static_cast<int32_t>(row0), 4 * kb);
             tma_load_2d(smem_u32(slot + kSlotRawB), &p.tmSB, fullsc_bar(s), nb * P_BN, 4 * kb);
           } else {
-            mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz : 0u) + b_sc_bytes);
-            if (a_sc) bulk_load(smem_u32(slot + kSlotRawA), ga + kb * p.sa_stride_k * esz, 128u * esz, fullsc_bar(s));
-            if (B_ROW) bulk_load(smem_u32(slot + kSlotRawB), gb + kb * p.sb_stride_k * esz, b_sc_bytes, fullsc_bar(s));
+            mbar_arrive_expect_tx(fullsc_bar(s), (a_sc ? 128u * esz_a : 0u) + b_sc_bytes);
+            if (a_sc) bulk_load(smem_u32(slot + dst_a), ga + kb * p.sa_stride_k * esz_a, 128u * esz_a, fullsc_bar(s));
+            if (B_ROW) bulk_load(smem_u32(slot + dst_b), gb + kb * p.sb_stride_k * esz_b, b_sc_bytes, fullsc_bar(s));
           }
         }
         __syncwarp();
@@ -901,11 +916,12 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       int mb, nb;
       tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
       uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
+      const bool sb_fp32 = kFp32 && !p.b_u8;  // B's block scales stored as FP32
       if (!B_ROW) {
         // lane l holds K block (kb0 rounded down to 32) + l, then the next 32
         const int base = u.kb0 & ~31;
-        load_block_scales(p, nb, base, kFp32, cur0, cur1);
-        load_block_scales(p, nb, base + 32, kFp32, nxt0, nxt1);
+        load_block_scales(p, nb, base, sb_fp32, cur0, cur1);
+        load_block_scales(p, nb, base + 32, sb_fp32, nxt0, nxt1);
       }
       for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
         const int s = it % P_STAGES;
@@ -913,7 +929,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         if (!B_ROW && kb > u.kb0 && (kb & 31) == 0) {
           cur0 = nxt0;
           cur1 = nxt1;
-          load_block_scales(p, nb, kb + 32, kFp32, nxt0, nxt1);
+          load_block_scales(p, nb, kb + 32, sb_fp32, nxt0, nxt1);
         }
         if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), ph, guard, kTimeoutScale))) { ok = false; break; }
         uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
@@ -924,8 +940,22 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         }
         if (kFp32) {
           if (!B_ROW && lane == 0) {
-            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[0] = b0;
-            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[1] = b1;
+            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[0] = p.b_u8 ? ue8m0_to_f32_bits(b0) : b0;
+            reinterpret_cast<uint32_t*>(slot + kSlotBlk)[1] = p.b_u8 ? ue8m0_to_f32_bits(b1) : b1;
+          }
+          // a mixed pair: the UE8M0 operand's raw scale bytes, decoded into
+          // the FP32 scale vectors the epilogue reads
+          if (p.a_u8) {
+            const uint8_t* raw = slot + kSlotTm;
+            uint32_t* f = reinterpret_cast<uint32_t*>(slot + kSlotRawA);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) f[32 * j + lane] = ue8m0_to_f32_bits(raw[32 * j + lane]);
+          }
+          if (B_ROW && p.b_u8) {
+            const uint8_t* raw = slot + kSlotTm + 128;
+            uint32_t* f = reinterpret_cast<uint32_t*>(slot + kSlotRawB);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[32 * j + lane] = ue8m0_to_f32_bits(raw[32 * j + lane]);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(sfready_bar(s));
@@ -1083,7 +1113,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             if (lane == 0) {
               bulk_wait_group0();
               fence_proxy_async_global();
-              st_release_gpu(p.ws_flag + 16 * cl + sub, 1);
+              if (cl != p.withhold_cluster) st_release_gpu(p.ws_flag + 16 * cl + sub, 1);
             }
             __syncwarp();
             continue;
@@ -1560,6 +1590,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
 __device__ int g_device_status;
 
 struct DeviceInfo {
+  unsigned long long ctx = 0;  // context the cached addresses and attributes belong to
   int sms = 0;
   int* status = nullptr;
   bool attr_set[8] = {};
@@ -1592,13 +1623,25 @@ cudaError_t device_info(DeviceInfo** out) {
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceInfo& d = g_dev[dev];
-  if (d.sms == 0) {
+  // The status word's address and the kernels' attributes belong to one
+  // context: a new context on this device (after cudaDeviceReset, say) is
+  // set up again.
+  const unsigned long long id = current_context_id();
+  if (d.sms == 0 || id == 0 || d.ctx != id) {
+    d = DeviceInfo{};
     e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      d.sms = 0;
+      return e;
+    }
     void* sym = nullptr;
-    e = cudaGetSymbolAddress(&sym, g_device_status);
-    if (e != cudaSuccess) return e;
+    e = cudaGetSymbolAddress(&sym, g_device_status);  // makes the device's context current if none is
+    if (e != cudaSuccess) {
+      d.sms = 0;
+      return e;
+    }
     d.status = static_cast<int*>(sym);
+    d.ctx = current_context_id();
   }
   *out = &d;
   return cudaSuccess;
@@ -1773,7 +1816,14 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
     *unsupported = true;
     return cudaSuccess;
   }
-  const bool pair = fused || mx || acc || pr.M > 128;
+  // a mixed pair (one operand's scales UE8M0, the other's FP32) decodes the
+  // UE8M0 bytes in the CTA-pair kernel's scale staging
+  const bool mixed = pr.a_u8 || pr.b_u8;
+  if (mixed && (fused || mx || pr.fmt != kFmtFp32)) {
+    *unsupported = true;
+    return cudaSuccess;
+  }
+  const bool pair = fused || mx || acc || mixed || pr.M > 128;
   Params prm;
   memset(&prm, 0, sizeof(prm));
   if (fused) {
@@ -1848,7 +1898,10 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.num_kb = static_cast<int>(pr.K / BK);
   prm.dp_tiles = prm.num_tiles;  // nothing split unless the pair launcher splits
   prm.status = di->status;
-  prm.limit_ns = 2000000000ull;  // 2 s per wait
+  prm.limit_ns = pr.wait_limit_ns != 0 ? pr.wait_limit_ns : 2000000000ull;  // 2 s per wait
+  prm.a_u8 = pr.a_u8 ? 1 : 0;
+  prm.b_u8 = pr.b_u8 ? 1 : 0;
+  prm.withhold_cluster = pr.withhold_cluster;
   const int grid = prm.num_tiles < di->sms ? prm.num_tiles : di->sms;
 
   const bool fp32 = pr.fmt == kFmtFp32;

@@ -6,7 +6,21 @@
 
 #include <cstdint>
 
+#include "fp8bq.h"
+
 namespace fp8bq {
+
+// FP8BQ_OK for cudaSuccess; otherwise records `e` as this thread's last CUDA
+// error (what fp8bq_last_cuda_error() returns) and gives FP8BQ_ERR_CUDA.
+// Every entry point maps its CUDA failures through this one function.
+int cuda_status(cudaError_t e);
+
+// Unique identifier of the CUDA context current on the calling thread
+// (cuCtxGetId: never reused within the process, unlike the context handle),
+// or 0 when no context is current or the driver entry point is missing.
+// Device addresses of the library's __device__ objects and per-function
+// attributes belong to one context; caches of them are keyed on this.
+unsigned long long current_context_id();
 
 inline int64_t round_up128(int64_t r) { return (r + 127) / 128 * 128; }
 
@@ -50,11 +64,27 @@ struct GemmProblem {
   GemmOperand a, b;
   void* d;
   int64_t M, N, K, ldd;
-  int fmt;        // kFmtFp32 / kFmtUe8m0 (both operands)
+  // Kernel family: kFmtUe8m0 (both operands UE8M0: block-scaled MMA) or
+  // kFmtFp32 (promotion path: at least one operand has FP32 scales; an
+  // operand with UE8M0 scales then has them decoded to 2^e, a_u8 / b_u8).
+  int fmt;
+  bool a_u8 = false, b_u8 = false;
   bool acc_f32;   // D is FP32 and accumulated into (D += A B^T); else BF16 D = A B^T
   void* ws = nullptr;    // split-tile workspace (flags zero between calls), or none
   int64_t ws_bytes = 0;
+  // Test hooks, off in every product call: the split-tile piece of this CTA
+  // pair stores its partial sum but never raises its flags (-1: none), and
+  // the bounded waits' limit in ns (0: the default 2 s).
+  int withhold_cluster = -1;
+  uint64_t wait_limit_ns = 0;
 };
+
+// Checks the arguments of fp8bq_gemm_ws (all but the workspace) and the
+// device, and fills `p`; returns FP8BQ_OK or the call's error status.
+int validate_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N, int64_t K,
+                  int64_t ldd, uint32_t flags, GemmProblem* p);
+// Launches a validated problem; returns a status.
+int run_gemm(const GemmProblem& p, cudaStream_t stream);
 
 // Split-tile workspace: one slot of a 256 x 256 FP32 partial sum per CTA
 // pair, then 16 int flags per slot (one per epilogue warp slice of the pair).

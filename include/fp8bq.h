@@ -38,7 +38,9 @@
  *     all-zero group), q = E4M3_RNE_satfinite(x * 2^-e).
  *   - Return value: FP8BQ_OK or one of the negative FP8BQ_ERR_* codes.  A call
  *     that returns an error has launched no kernel and written no caller
- *     memory (fp8bq_gemm_noalloc may have cleared its own array's flags).
+ *     memory.  (The one exception: when fp8bq_gemm_noalloc's launch itself
+ *     fails with ERR_CUDA, the clearing of its own array's flags has
+ *     already been queued; argument errors queue nothing.)
  */
 #ifndef FP8BQ_H
 #define FP8BQ_H
@@ -88,7 +90,12 @@ typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
  *            FP8BQ_GRAN_BLOCK_128x128 (B only), or FP8BQ_GRAN_ROW_1x32 (MX:
  *            A and B both, k_major, UE8M0; the weight is quantized in 1x32
  *            groups along its contraction like an activation).
- *   fmt      FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0; A and B must agree.
+ *   fmt      FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0, per operand.  Both
+ *            UE8M0: the block-scaled MMA.  Otherwise (both FP32, or a mixed
+ *            pair) the per-128-K promotion path, in which a UE8M0 operand's
+ *            scale bytes are decoded to the FP32 value 2^e as they are
+ *            staged; the product is the same definition either way.  A BF16
+ *            A is quantized in its own fmt and B must then have the same.
  *   s_stride_k, s_stride_r
  *            the scale of element (r, k) is scales[(k/G)*s_stride_k +
  *            t*s_stride_r], t = r (row groups) or t = r/128 (blocks), G = 32
@@ -248,8 +255,10 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
  *   dgrad    A = quantize_act(dY), B = W^T (k_major = 0)        D = dX [M, K_w]
  *   wgrad    A = quantize_act_t(dY), B = quantize_act_t(X)      D = dW [N, K]
  * FP32 scales run the per-128-K promotion path (partial products in tensor
- * memory, rescaled into FP32 accumulators); UE8M0 scales run the block-scaled
- * MMA (MXFP8 route).
+ * memory, rescaled into FP32 accumulators); UE8M0 scales on both operands run
+ * the block-scaled MMA (MXFP8 route); a mixed pair (one operand FP32, the
+ * other UE8M0: DeepSeek-V3-style blocks meeting MXFP8 ones) runs the
+ * promotion path with the UE8M0 scales decoded to 2^e.
  *   D       BF16 [M, N], leading dimension ldd (ldd >= N, ldd % 8 == 0); FP32
  *           with FP8BQ_GEMM_ACCUMULATE_F32.
  *   K       contraction length, K % 128 == 0, K > 0.
@@ -263,9 +272,10 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
  *           ERR_INVALID_ARG.
  * Errors: ERR_INVALID_ARG, ERR_SHAPE (M,N <= 0, K % 128 != 0, N % 8 != 0),
  * ERR_ALIGN (a pointer not 16-B aligned, a leading dimension not a multiple
- * of 16 bytes), ERR_UNSUPPORTED (mixed scale formats, BF16 B, row-group B
- * that is not k-major, MX operands mixed with other granularities or not
- * both k-major UE8M0), ERR_CUDA (tensor-map encoding or launch failed).
+ * of 16 bytes), ERR_UNSUPPORTED (BF16 B, a BF16 A whose fmt differs from
+ * B's, row-group B that is not k-major, MX operands mixed with other
+ * granularities or not both k-major UE8M0), ERR_CUDA (tensor-map encoding or
+ * launch failed).
  */
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
                int64_t K, int64_t ldd, uint32_t flags, fp8bq_stream_t stream);
@@ -321,10 +331,13 @@ int64_t fp8bq_gemm_workspace_bytes(void);
  *   that loads the library until the process exits); on a device with more
  *   than 160 multiprocessors the call returns ERR_UNSUPPORTED.  Nothing is
  *   allocated: no cudaMalloc, no cudaFree.
- *   The first call on each device looks up the array's device address with
- *   that device current (cudaGetSymbolAddress); make that first call before
- *   any stream capture.  Every call then clears the array's flag words on
- *   the stream (cudaMemsetAsync) before the GEMM.
+ *   The first call in each CUDA context (on each device, and again after a
+ *   cudaDeviceReset) looks up the array's device address with that device
+ *   current (cudaGetSymbolAddress); make that first call before any stream
+ *   capture.  Every call checks all its arguments first (an argument error
+ *   queues nothing), then clears the array's flag words on the stream
+ *   (cudaMemsetAsync) before the GEMM; with FP8BQ_GEMM_ACCUMULATE_F32,
+ *   which splits nothing, the array is not touched.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: calls that may overlap on the GPU (other streams, other host
  *   threads) race on it and must be ordered by the caller.

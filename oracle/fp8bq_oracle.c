@@ -387,6 +387,18 @@ void oracle_gemm(const oracle_operand* A, const oracle_operand* B, int64_t C,
   }
 }
 
+/* The weight gradient added into an FP32 master gradient (the digest's
+ * "方法": master weights and optimizer state stay in FP32): out[i][j] =
+ * d0[rows[i]][cols[j]] + the product above, in float64.  d0 is the FP32
+ * gradient before the call, row-major with leading dimension ldd0. */
+void oracle_gemm_accumulate(const oracle_operand* A, const oracle_operand* B, int64_t C,
+                            const int64_t* rows, int64_t nr, const int64_t* cols, int64_t nc,
+                            const float* d0, int64_t ldd0, double* out) {
+  oracle_gemm(A, B, C, rows, nr, cols, nc, out);
+  for (int64_t i = 0; i < nr; i++)
+    for (int64_t j = 0; j < nc; j++) out[i * nc + j] += (double)d0[rows[i] * ldd0 + cols[j]];
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

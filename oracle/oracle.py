@@ -2,7 +2,8 @@
 
 Inputs and outputs are numpy arrays on the host.  BF16 tensors travel as their
 uint16 bit patterns.  Nothing here computes any part of the method: every
-number comes from the C file, which states the definition it follows.
+number comes from the C file, which states the definition it follows; this
+module only allocates the outputs and passes pointers and indices.
 """
 from __future__ import annotations
 
@@ -71,6 +72,10 @@ def lib():
         L.oracle_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), ctypes.c_int64,
                                   ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
                                   ctypes.c_void_p]
+        L.oracle_gemm_accumulate.restype = None
+        L.oracle_gemm_accumulate.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_int64,
+                                             ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p]
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_swiglu.restype = None
         L.oracle_swiglu.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
@@ -117,13 +122,19 @@ def gemm_accumulate(A: "Operand", B: "Operand", d0: np.ndarray, rows=None, cols=
     added into an FP32 master gradient (the Puro-2B digest, section "方法": master
     weights and optimizer state stay in FP32).  d0 is the FP32 gradient before
     the call, [A.rows, B.rows]."""
-    g = gemm(A, B, rows, cols)
-    d = np.asarray(d0, np.float64)
-    if rows is not None:
-        d = d[np.asarray(rows, np.int64)]
-    if cols is not None:
-        d = d[:, np.asarray(cols, np.int64)]
-    return d + g
+    C = A.contraction
+    if B.contraction != C:
+        raise ValueError("contraction mismatch")
+    d = np.ascontiguousarray(d0, np.float32)
+    if d.shape != (A.rows, B.rows):
+        raise ValueError("d0 must be [A.rows, B.rows]")
+    r = np.arange(A.rows, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    c = np.arange(B.rows, dtype=np.int64) if cols is None else np.ascontiguousarray(cols, dtype=np.int64)
+    out = np.empty((r.size, c.size), np.float64)
+    ca, cb = A._c(), B._c()
+    lib().oracle_gemm_accumulate(ctypes.byref(ca), ctypes.byref(cb), C, r.ctypes.data, r.size, c.ctypes.data,
+                                 c.size, d.ctypes.data, d.shape[1], out.ctypes.data)
+    return out
 
 
 def num_threads() -> int:

@@ -1,6 +1,7 @@
 """The C-ABI boundary on the CPU: libfp8bq.so loads, exports every function
-include/fp8bq.h declares, and rejects bad arguments with the documented status
-codes before it touches a device (fake pointers are never dereferenced)."""
+the headers under include/ declare, and rejects bad arguments with the
+documented status codes before it touches a device (fake pointers are never
+dereferenced)."""
 import ctypes
 import os
 import re
@@ -22,14 +23,19 @@ def L():
 
 
 def declared_functions():
-    src = open(os.path.join(ROOT, "include", "fp8bq.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fp8bq_[a-z0-9_]+)\s*\(", src)))
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for h in sorted(os.listdir(inc)):
+        if h.endswith(".h"):
+            src = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, h)).read(), flags=re.S)
+            names.update(re.findall(r"\b(fp8bq_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_function(L):
     names = declared_functions()
     assert "fp8bq_gemm" in names and "fp8bq_quantize_act_t" in names
+    assert "fp8bq_testing_gemm_ws_withhold" in names and "fp8bq_gemm_noalloc" in names
     for n in names:
         assert hasattr(L, n), n
 
@@ -160,8 +166,14 @@ def test_gemm_argument_checks(L):
     assert g(_op(L, s_stride_r=2), B) == SHAPE
     assert g(_op(L, dtype=5), B) == INVALID
     assert g(_op(L, gran=3), B) == INVALID
-    assert g(_op(L, fmt=1), B) == UNSUPPORTED or g(_op(L, fmt=1), B) == INVALID  # mixed formats
-    assert g(A, _op(L, gran=1, s_stride_k=1, s_stride_r=1, fmt=1)) == UNSUPPORTED
+    assert g(_op(L, fmt=2), B) == INVALID          # unknown scale format
+    # a mixed pair (UE8M0 A, FP32 B or the reverse) passes every argument check
+    # and runs the promotion path; here it then finds no device
+    assert g(_op(L, fmt=1), B) in (CUDA, UNSUPPORTED)
+    assert g(A, _op(L, gran=1, s_stride_k=2, s_stride_r=1, fmt=1)) in (CUDA, UNSUPPORTED)
+    # a BF16 A is quantized in its own format: B must share it
+    assert g(_op(L, dtype=1, scales=0, ld=512, fmt=0), _op(L, gran=1, s_stride_k=2, s_stride_r=1, fmt=1)) == UNSUPPORTED
+    assert g(A, _op(L, gran=1, s_stride_k=1, s_stride_r=1, fmt=1)) == SHAPE  # W^T block strides too short
     assert g(_op(L, gran=1, s_stride_k=4, s_stride_r=1), B) == UNSUPPORTED  # block-scaled A
     assert g(A, _op(L, k_major=0, ld=256)) == UNSUPPORTED   # row-group B must be k-major
     assert g(A, _op(L, gran=1, s_stride_k=3, s_stride_r=3)) == SHAPE  # neither layout
@@ -183,9 +195,38 @@ def test_gemm_noalloc_argument_checks(L):
     f = L.fp8bq_gemm_noalloc
     A = _op(L)
     B = _op(L, gran=1, s_stride_k=2, s_stride_r=1)
-    assert f(None, ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == INVALID
-    assert f(ctypes.byref(A), ctypes.byref(B), None, 256, 256, 512, 256, 0, None) == INVALID
-    assert f(ctypes.byref(A), ctypes.byref(B), P, 256, 256, 512, 256, 0, None) == UNSUPPORTED  # no device here
+    g = lambda A_, B_, D=P, k=512, flags=0: f(ctypes.byref(A_) if A_ is not None else None, ctypes.byref(B_), D,
+                                              256, 256, k, 256, flags, None)
+    # every argument is checked before anything is queued, as fp8bq_gemm checks them
+    assert g(None, B) == INVALID
+    assert g(A, B, D=None) == INVALID
+    assert g(A, B, k=100) == SHAPE
+    assert g(A, B, D=P + 8) == ALIGN
+    assert g(A, B, flags=2) == INVALID
+    assert g(_op(L, gran=1, s_stride_k=4, s_stride_r=1), B) == UNSUPPORTED
+    # valid arguments: no device here, which the call reports as a CUDA error
+    # and records for fp8bq_last_cuda_error()
+    L.fp8bq_last_cuda_error.restype = ctypes.c_int
+    assert g(A, B) == CUDA
+    assert L.fp8bq_last_cuda_error() != 0
+
+
+def test_testing_hook_argument_checks(L):
+    f = L.fp8bq_testing_gemm_ws_withhold
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int64,
+                  ctypes.c_void_p]
+    A = _op(L)
+    B = _op(L, gran=1, s_stride_k=2, s_stride_r=1)
+    g = lambda ws=P, nbytes=1 << 24, pair=0, limit=1000000: f(ctypes.addressof(A), ctypes.addressof(B), P, 256, 256,
+                                                              512, 256, 0, ws, nbytes, pair, limit, None)
+    assert g(ws=None) == INVALID              # the hook needs a workspace
+    assert g(pair=-1) == INVALID
+    assert g(limit=10) == INVALID             # below 100 us
+    assert g(limit=3 * 10 ** 9) == INVALID    # above the product's 2 s
+    assert g(ws=P + 16) == ALIGN
+    assert g() in (CUDA, UNSUPPORTED)         # valid: no device here
 
 
 def test_swiglu_quantize_argument_checks(L):

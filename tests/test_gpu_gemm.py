@@ -209,6 +209,25 @@ def test_mlp_backward_full_size(fmt):
                     nrows=8, ncols=8, nelem=1024)
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("lin", [l for l in synth.layer_linears(16384) if l.name != "gate_up"], ids=lambda l: l.name)
+def test_dgrad_full_size(fmt, lin):
+    """The data gradients of the QKV, O and down projections at M = 16384
+    tokens, dX [M, K] = dY [M, N] W [N, K] with W's 128x128 blocks read
+    transposed in place, launched as the benchmark launches them (with a
+    split-tile workspace); sampled against the oracle."""
+    dy = lin.dy(4400, device="cuda")
+    w = lin.w(4400, device="cuda")
+    qw, sw = fp.quantize_weight(w, fmt)
+    qd, sd = fp.quantize_act(dy, fmt)
+    del dy, w
+    dX = fp.gemm(fp.row_operand(qd, sd, fmt), fp.block_operand(qw, sw, fmt, transposed=True),
+                 workspace=fp.gemm_workspace())
+    assert dX.shape == (lin.M, lin.K)
+    compare_sampled(dX, o_row(qd, sd, fmt), o_block(qw, sw, fmt, transposed=True), f"{lin.name} dgrad",
+                    nrows=8, ncols=8, nelem=1024, seed=4400)
+
+
 def test_no_pending_device_error():
     fp.check()
 
