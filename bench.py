@@ -61,8 +61,15 @@ def measured_peaks():
     try:
         with open(path) as f:
             p = json.load(f)
-        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
-                "bf16_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+        out = {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+               "bf16_sustained": float(p["bf16_tflops_sustained"]), "source": "measured"}
+        # the SM clock the burst peak was measured at, where the file gives one
+        for key in ("bf16_sm_mhz", "bf16_clock_mhz", "sm_mhz_burst", "burst_sm_mhz"):
+            if isinstance(p.get(key), (int, float)):
+                out["sm_mhz"] = float(p[key])
+                break
+        out["keys"] = sorted(p.keys())
+        return out
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
@@ -134,10 +141,12 @@ class ClockSampler:
 class LayerStep:
     """Device buffers and the launch sequence of one step."""
 
-    def __init__(self, fp, fmt, seed, device, only=None, dual=True, mx=False, split=True):
+    def __init__(self, fp, fmt, seed, device, only=None, dual=True, mx=False, split=True, group=True):
         self.fp = fp
         self.fmt = fmt
         self.dual = dual
+        # the forward's input (both layouts) and the weight in one grouped launch
+        self.group = group and dual and not mx
         # GEMM workspace: the last round of output tiles may be split along K
         self.ws = fp.gemm_workspace(device) if split else None
         self.mx = mx  # 1x32 MX blocks (UE8M0) on every operand; weights quantized in both orientations
@@ -204,6 +213,8 @@ class LayerStep:
     def launches(self):
         if self.mx:
             return 7 * len(self.items)
+        if self.group:
+            return 5 * len(self.items)
         return (6 if self.dual else 8) * len(self.items)
 
     def run(self, ev=None, external=False):
@@ -243,11 +254,16 @@ class LayerStep:
                                               fp.mx_operand(it["qxt"], it["sxt"]), it["dw"], workspace=self.ws))
             return
         for it in self.items:
-            if self.dual:
+            if self.group:
+                timed("quant", lambda: fp.quantize_group(
+                    [("dual", it["x"], (it["qx"], it["sx"], it["qxt"], it["sxt"])), ("weight", it["w"], (it["qw"], it["sw"]))],
+                    f))
+            elif self.dual:
                 timed("quant", lambda: fp.quantize_act_dual(it["x"], f, it["qx"], it["sx"], it["qxt"], it["sxt"]))
             else:
                 timed("quant", lambda: fp.quantize_act(it["x"], f, it["qx"], it["sx"]))
-            timed("quant", lambda: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
+            if not self.group:
+                timed("quant", lambda: fp.quantize_weight(it["w"], f, it["qw"], it["sw"]))
             timed("gemm", lambda: fp.gemm(fp.row_operand(it["qx"], it["sx"], f),
                                           fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=self.ws))
             if self.dual:
@@ -268,17 +284,10 @@ def l2_flush(buf):
     buf.zero_()
 
 
-def run_ours(args, rank, world, dist):
-    import blockwise_fp8_linear_fp8bq_b200 as fp
-    fp.lib()
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
-    torch.cuda.set_device(dev)
-    fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
-    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant,
-                     mx=args.scale == "mx", split=not args.no_split)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
-
+def measure_step(args, fp, step, dev, dist, flush):
+    """Warm up, then time `args.steps` steps of `step` as two CUDA graphs (see
+    below).  Returns step / kernel-split times, the NVML clock records of both
+    replays, and the SM clock the GEMM kernels themselves counted."""
     for _ in range(args.warmup):
         step.run()
     fp.check()
@@ -290,10 +299,14 @@ def run_ours(args, rank, world, dist):
     # first, which adds an event between every two launches; those
     # event-record nodes order the kernels strictly, so its step runs a few
     # percent longer.  The host's Python and ctypes work is outside both.  (--no-graph
-    # issues the same two sequences eagerly.)
+    # issues the same two sequences eagerly.)  The GEMMs of the kernel-split
+    # graph also add up their SM cycles and nanoseconds (clock counters): the
+    # clock the tensor cores ran at, which NVML's 5 ms samples do not resolve.
     step_events, split_step_events, kernel_events = [], [], []
+    clk = torch.zeros(2, dtype=torch.int64, device=dev)
 
     def timed_steps(per_launch, external):
+        fp.set_clock_counters(clk if per_launch else None)
         for _ in range(args.steps):
             l2_flush(flush)
             a = torch.cuda.Event(enable_timing=True, external=external)
@@ -302,6 +315,7 @@ def run_ours(args, rank, world, dist):
             step.run(kernel_events if per_launch else None, external=external)
             b.record()
             (split_step_events if per_launch else step_events).append((a, b))
+        fp.set_clock_counters(None)
 
     graphs = {}
     if not args.no_graph:
@@ -331,17 +345,38 @@ def run_ours(args, rank, world, dist):
             dist.barrier()
         return sampler.stop()
 
+    clk.zero_()
     clocks_split = replay(True)
+    cyc, ns = (int(v) for v in clk.tolist())
     # idle between the two replays, so that the second starts from the power
     # state the first did rather than from the end of a 70 ms burst
     time.sleep(2.0)
     clocks = replay(False)
     fp.check()
-    step_ms = sum(a.elapsed_time(b) for a, b in step_events)
-    split_step_ms = sum(a.elapsed_time(b) for a, b in split_step_events)
-    gemm_ms = sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "gemm")
-    quant_ms = sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "quant")
     graphs.clear()
+    return dict(step_ms=sum(a.elapsed_time(b) for a, b in step_events),
+                split_step_ms=sum(a.elapsed_time(b) for a, b in split_step_events),
+                gemm_ms=sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "gemm"),
+                quant_ms=sum(a.elapsed_time(b) for k, a, b in kernel_events if k == "quant"),
+                clocks=clocks, clocks_split=clocks_split,
+                gemm_kernel_mhz=(1e3 * cyc / ns) if ns > 0 else None,
+                gemm_launches=len([1 for k, _, _ in kernel_events if k == "gemm"]),
+                quant_launches=len([1 for k, _, _ in kernel_events if k == "quant"]))
+
+
+def run_ours(args, rank, world, dist):
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    fp.lib()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    fmt = fp.SCALE_FP32 if args.scale == "fp32" else fp.SCALE_UE8M0
+    step = LayerStep(fp, fmt, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant,
+                     mx=args.scale == "mx", split=not args.no_split, group=not args.no_group_quant)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20) // 4, dtype=torch.float32, device=dev)
+    m = measure_step(args, fp, step, dev, dist, flush)
+    step_ms, split_step_ms, gemm_ms, quant_ms = m["step_ms"], m["split_step_ms"], m["gemm_ms"], m["quant_ms"]
+    clocks, clocks_split = m["clocks"], m["clocks_split"]
 
     # end to end: every step's inputs (X, W, dY of the four linears) copied
     # from pinned host memory and its outputs (Y, dX, dW) copied back inside
@@ -414,11 +449,193 @@ def run_ours(args, rank, world, dist):
         e2e = {"ms_per_step": e2e_ms, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo, "steps": e2e_steps,
                "copies": "one stream per PCIe direction, overlapped with the step's kernels"}
 
-    return dict(step_ms=step_ms, split_step_ms=split_step_ms, gemm_ms=gemm_ms, quant_ms=quant_ms,
-                clocks=clocks, clocks_split=clocks_split, e2e=e2e,
-                flops=step.gemm_flops(), qbytes=step.quant_bytes(), launches=step.launches() * args.steps,
-                gemm_launches=len([1 for k, _, _ in kernel_events if k == "gemm"]),
-                quant_launches=len([1 for k, _, _ in kernel_events if k == "quant"]))
+    out = dict(step_ms=step_ms, split_step_ms=split_step_ms, gemm_ms=gemm_ms, quant_ms=quant_ms,
+               clocks=clocks, clocks_split=clocks_split, e2e=e2e, gemm_kernel_mhz=m["gemm_kernel_mhz"],
+               flops=step.gemm_flops(), qbytes=step.quant_bytes(), launches=step.launches() * args.steps,
+               gemm_launches=m["gemm_launches"], quant_launches=m["quant_launches"])
+    extras = world == 1 and args.scale == "ue8m0"
+    # the same step with FP32 scales (the DeepSeek-V3-style promotion path),
+    # measured the same way, as a sub-record of the default line
+    if extras and not args.no_fp32_record:
+        step32 = LayerStep(fp, fp.SCALE_FP32, seed=1000 * (rank + 1), device=dev, dual=not args.separate_quant,
+                           split=not args.no_split, group=not args.no_group_quant)
+        time.sleep(2.0)
+        m32 = measure_step(args, fp, step32, dev, dist, flush)
+        out["fp32"] = dict(m32, flops=step32.gemm_flops(), qbytes=step32.quant_bytes())
+        del step32
+        torch.cuda.empty_cache()
+    # the 28-layer sweep plus the LM head, end to end (quantizers + GEMMs)
+    if extras and not args.no_sweep:
+        time.sleep(2.0)
+        out["sweep"] = run_sweep(args, fp, step, dev, flush)
+    if extras:
+        out["fp8_ceiling"] = fp8_cublas_ceiling(dev)
+    return out
+
+
+# ------------------------------------------------------------ the sweep --
+SWEEP_LAYERS = 28
+
+
+def sweep_flops(M=M_TOKENS):
+    return SWEEP_LAYERS * sum(3 * lin.flops for lin in linears(M)) + synth.LM_HEAD.flops
+
+
+def run_sweep(args, fp, step, dev, flush, reps=3):
+    """The full 28-layer linear sweep with an untied LM head: per layer the
+    four linears' forward, dgrad and wgrad with their quantizers (each layer
+    its own seeded inputs X, W, dY), then the LM head's weight and input
+    quantization and its forward GEMM [16384 x 2048] . [151936 x 2048]^T.
+    End to end on the device (quantizers + GEMMs, 562 launches), one CUDA
+    graph replayed `reps` times after an L2 flush each; the LM head's output
+    is then checked on sampled rows, columns and elements."""
+    fmt = step.fmt
+    per_layer = []
+    for layer in range(1, SWEEP_LAYERS):
+        bufs = []
+        for i, it in enumerate(step.items):
+            lin = it["lin"]
+            s = 90000 + 1000 * layer + 100 * i
+            bufs.append(dict(x=lin.x(s, device=dev), w=lin.w(s, device=dev), dy=lin.dy(s, device=dev)))
+        per_layer.append(bufs)
+    per_layer.insert(0, [dict(x=it["x"], w=it["w"], dy=it["dy"]) for it in step.items])
+    lm = synth.LM_HEAD
+    x_lm, w_lm = lm.x(95000, device=dev), lm.w(95000, device=dev)
+    sdt = torch.float32 if fmt == fp.SCALE_FP32 else torch.uint8
+    qx_lm = torch.empty(lm.M, lm.K, dtype=torch.float8_e4m3fn, device=dev)
+    sx_lm = torch.empty(lm.K // 128, fp.row_scale_ld(lm.M), dtype=sdt, device=dev)
+    qw_lm = torch.empty(lm.N, lm.K, dtype=torch.float8_e4m3fn, device=dev)
+    sw_lm = torch.empty(lm.K // 128, (lm.N + 127) // 128, dtype=sdt, device=dev)
+    y_lm = torch.empty(lm.M, lm.N, dtype=torch.bfloat16, device=dev)
+    A_lm, B_lm = fp.row_operand(qx_lm, sx_lm, fmt), fp.block_operand(qw_lm, sw_lm, fmt)
+
+    def one_sweep():
+        for bufs in per_layer:
+            for it, b in zip(step.items, bufs):
+                it["x"], it["w"], it["dy"] = b["x"], b["w"], b["dy"]
+            step.run()
+        fp.quantize_group([("act", x_lm, (qx_lm, sx_lm)), ("weight", w_lm, (qw_lm, sw_lm))], fmt)
+        fp.gemm(A_lm, B_lm, y_lm, workspace=step.ws)
+
+    one_sweep()  # warm-up, and every operand produced once
+    fp.check()
+    events = []
+    g = torch.cuda.CUDAGraph()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        l2_flush(flush)
+        a = torch.cuda.Event(enable_timing=True, external=True)
+        b = torch.cuda.Event(enable_timing=True, external=True)
+        a.record()
+        one_sweep()
+        b.record()
+        events.append((a, b))
+    torch.cuda.synchronize()
+    times = []
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(reps):
+        g.replay()
+        torch.cuda.synchronize()
+        times.append(events[0][0].elapsed_time(events[0][1]))
+    clocks = sampler.stop()
+    fp.check()
+    del g
+    # restore the layer-0 inputs the step buffers held
+    for it, b in zip(step.items, per_layer[0]):
+        it["x"], it["w"], it["dy"] = b["x"], b["w"], b["dy"]
+    check = lm_head_check(fp, fmt, qx_lm, sx_lm, qw_lm, sw_lm, y_lm)
+    ms = statistics.median(times)
+    flops = sweep_flops()
+    del per_layer, x_lm, w_lm, y_lm
+    torch.cuda.empty_cache()
+    return {"layers": SWEEP_LAYERS, "ms": ms, "ms_all": times, "tflops": flops / (ms * 1e-3) / 1e12,
+            "flops": flops, "launches": SWEEP_LAYERS * step.launches() + 2, "clocks": clocks,
+            "lm_head_check": check,
+            "what": "28 layers x (qkv, o, gate_up, down) x (fwd, dgrad, wgrad) with their quantizers at M=16384, "
+                    "then the LM head weight + input quantization and forward GEMM; one graph replay per sweep, "
+                    "L2 flushed before each"}
+
+
+def _dequant_rows(q: torch.Tensor, s: torch.Tensor, fmt: int, rows: torch.Tensor) -> torch.Tensor:
+    """float64 values of 1x128-group codes q[rows] (scales [K/128][ld])."""
+    v = q[rows].float().double()
+    sc = s[:, rows].t()
+    sc = sc.to(torch.float64) if sc.dtype == torch.float32 else torch.exp2(sc.to(torch.float64) - 127.0)
+    return v * sc.repeat_interleave(128, dim=1)
+
+
+def _dequant_block_rows(q: torch.Tensor, s: torch.Tensor, rows: torch.Tensor) -> torch.Tensor:
+    """float64 values of 128x128-block codes q[rows] (scales [K/128][ceil(N/128)])."""
+    v = q[rows].float().double()
+    sc = s[:, rows // 128].t()
+    sc = sc.to(torch.float64) if sc.dtype == torch.float32 else torch.exp2(sc.to(torch.float64) - 127.0)
+    return v * sc.repeat_interleave(128, dim=1)
+
+
+def lm_head_check(fp, fmt, qx, sx, qw, sw, y, nrows=4, ncols=4, nelem=1024, seed=4242):
+    """The LM head output against the definition D = deq(A) deq(B)^T in
+    float64 (torch on the device), on sampled whole rows, whole columns and
+    single elements, with the tests' tolerance: relative Frobenius error
+    <= 5e-3 and |diff| <= 1e-2 rms + half a BF16 ulp per element."""
+    M, N = y.shape
+    dev = y.device
+    g = torch.Generator().manual_seed(seed)
+    rows = torch.randperm(M, generator=g)[:nrows].tolist() + [M - 1]
+    cols = torch.randperm(N, generator=g)[:ncols].tolist() + [N - 1]
+    er = torch.randint(0, M, (nelem,), generator=g)
+    ec = torch.randint(0, N, (nelem,), generator=g)
+    r_t, c_t = torch.tensor(rows, device=dev), torch.tensor(cols, device=dev)
+    xa = _dequant_rows(qx, sx, fmt, r_t)
+    ref_rows = torch.cat([xa @ _dequant_block_rows(qw, sw, torch.arange(n0, min(n0 + 16384, N), device=dev)).t()
+                          for n0 in range(0, N, 16384)], dim=1)
+    wb = _dequant_block_rows(qw, sw, c_t)
+    ref_cols = torch.cat([_dequant_rows(qx, sx, fmt, torch.arange(m0, min(m0 + 4096, M), device=dev)) @ wb.t()
+                          for m0 in range(0, M, 4096)], dim=0)
+    er_d, ec_d = er.to(dev), ec.to(dev)
+    ref_el = (_dequant_rows(qx, sx, fmt, er_d) * _dequant_block_rows(qw, sw, ec_d)).sum(dim=1)
+    got = torch.cat([y[r_t].double().ravel(), y[:, c_t].double().ravel(), y[er_d, ec_d].double()])
+    ref = torch.cat([ref_rows.ravel(), ref_cols.ravel(), ref_el])
+    diff = got - ref
+    rel = float(diff.norm() / ref.norm())
+    rms = float(ref.pow(2).mean().sqrt())
+    _, e = torch.frexp(ref.abs())
+    half_ulp = torch.ldexp(torch.ones_like(ref), (e - 9).to(torch.int32)) * (ref != 0)
+    excess = float((diff.abs() - (1e-2 * rms + half_ulp)).max())
+    return {"ok": rel <= 5e-3 and excess <= 0.0, "rel_frobenius": rel, "max_excess_over_bound": excess,
+            "values_checked": int(ref.numel()), "how": "sampled rows, columns and elements vs float64 torch "
+            "dequantize-then-matmul on the device"}
+
+
+def fp8_cublas_ceiling(dev, n=8192, reps=20):
+    """A measured FP8 ceiling beside the BF16 x 2 denominator: cuBLASLt's FP8
+    GEMM (torch._scaled_mm, E4M3 x E4M3 -> BF16, per-tensor scales) at
+    8192^3, timed with CUDA events after an L2 flush each.  A cross-check of
+    the denominator only; nothing of the path runs through it."""
+    try:
+        g = torch.Generator(device=dev).manual_seed(7)
+        a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        f = lambda: torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            f()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        ms = statistics.median(ts)
+        return {"tflops": 2.0 * n ** 3 / (ms * 1e-3) / 1e12, "ms": ms, "shape": f"{n}^3",
+                "what": "torch._scaled_mm (cuBLASLt FP8 e4m3, bf16 out), median of 20 after an L2 flush each"}
+    except Exception as exc:  # pragma: no cover - depends on the box's torch build
+        return {"unavailable": str(exc)[:200]}
 
 
 # --------------------------------------------------------- oracle on CPU --
@@ -558,6 +775,11 @@ def case_launchers(step, fp):
                                     lambda it=it: fp.quantize_act_dual(it["x"], f, it["qx"], it["sx"], it["qxt"], it["sxt"]))
         out[f"quant_dual:dy:{n}"] = ("quant", M * N * 4 + ((N // 128) * M + (M // 128) * N) * sb,
                                      lambda it=it: fp.quantize_act_dual(it["dy"], f, it["qd"], it["sd"], it["qdt"], it["sdt"]))
+        out[f"quant_group:x_w:{n}"] = ("quant", M * K * 4 + ((K // 128) * M + (M // 128) * K) * sb + N * K * 3
+                                       + (K // 128) * ((N + 127) // 128) * sb,
+                                       lambda it=it: fp.quantize_group(
+                                           [("dual", it["x"], (it["qx"], it["sx"], it["qxt"], it["sxt"])),
+                                            ("weight", it["w"], (it["qw"], it["sw"]))], f))
         out[f"gemm_fwd:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.row_operand(it["qx"], it["sx"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=step.ws))
         out[f"gemm_dgrad:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
@@ -688,6 +910,10 @@ def main(argv=None):
     ap.add_argument("--no-split", action="store_true",
                     help="GEMMs without a workspace: no output tiles split along K")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 28-layer + LM head sweep record")
+    ap.add_argument("--no-group-quant", action="store_true",
+                    help="quantize each linear's input and weight in separate launches instead of one grouped launch")
+    ap.add_argument("--no-fp32-record", action="store_true", help="skip the FP32-scale sub-record")
     ap.add_argument("--case", default=None,
                     help="time single kernels instead of the step: 'all' or a name such as gemm_fwd:gate_up")
     args = ap.parse_args(argv)
@@ -748,6 +974,8 @@ def main(argv=None):
         "config": {"workload": WORKLOAD, "scale_format": args.scale, "tokens": M_TOKENS,
                    "activation_quant": "separate act / act_t launches" if args.separate_quant
                    else "dual (one read of X and of dY, both code layouts)",
+                   "weight_quant": "grouped with the forward input (one launch per linear)"
+                   if not (args.no_group_quant or args.separate_quant or args.scale == "mx") else "own launch",
                    "launch": "eager" if args.no_graph else "CUDA graph of the timed steps",
                    "gemm_tiles": "whole tiles" if args.no_split else "last round split along K where it pays",
                    "parallelism": f"replicas{world}", "l2": "flushed between steps (write of 2x L2)"},
@@ -767,6 +995,40 @@ def main(argv=None):
         "kernel_split": {"source": "a replay, before the timed one, of the same K steps with an event between every two launches",
                          "ms_per_step": split_ms, "clocks": r["clocks_split"]},
     }
+    # the SM clock the GEMM kernels counted themselves (clock64 over
+    # globaltimer, summed over CTAs) during the kernel-split replay; the
+    # roofline against the burst peak scaled to that clock, taking the peak's
+    # own clock as the maximum NVML reports under a burst
+    kmhz = r.get("gemm_kernel_mhz")
+    if kmhz:
+        ref_mhz = peaks.get("sm_mhz") or (r["clocks"] or {}).get("sm_max_mhz") or 1965.0
+        out["roofline"]["gemm_kernel_sm_mhz"] = kmhz
+        out["roofline"]["peak_at_kernel_clock"] = fp8_peak * kmhz / ref_mhz
+        out["roofline"]["frac_at_kernel_clock"] = gemm_tflops / (fp8_peak * kmhz / ref_mhz)
+        out["roofline"]["peak_clock_mhz_assumed"] = ref_mhz
+    if r.get("fp8_ceiling"):
+        out["roofline"]["fp8_cublas_8192"] = r["fp8_ceiling"]
+    if r.get("fp32"):
+        f = r["fp32"]
+        g32 = f["flops"] * args.steps / (f["gemm_ms"] * 1e-3) / 1e12
+        q32 = f["qbytes"] * args.steps / (f["quant_ms"] * 1e-3) / 1e9
+        out["fp32_scales"] = {
+            "value": f["flops"] / (f["step_ms"] / args.steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": f["step_ms"] / args.steps,
+            "gemm": {"tflops": g32, "frac": g32 / fp8_peak, "frac_of_nominal_4500": g32 / 4500.0,
+                     "ms_per_step": f["gemm_ms"] / args.steps,
+                     "sm_mhz_in_kernel": f.get("gemm_kernel_mhz")},
+            "quantizers": {"achieved_gbs": q32, "frac": q32 / peaks["hbm_gbs"],
+                           "ms_per_step": f["quant_ms"] / args.steps},
+            "clocks": f["clocks"],
+            "what": "the same step with FP32 scales (per-128-K promotion in the epilogue), same seeds and timing"}
+    if r.get("sweep"):
+        sw = r["sweep"]
+        out["sweep"] = {"config": "28-layer Qwen3-1.7B linear sweep + untied LM head, M=16384 (end to end)",
+                        "value": sw["tflops"], "unit": "TFLOP/s", "ms": sw["ms"], "ms_all": sw["ms_all"],
+                        "tflop": sw["flops"] / 1e12, "frac": sw["tflops"] / fp8_peak, "launches": sw["launches"],
+                        "clocks": sw["clocks"], "lm_head_check": sw["lm_head_check"], "what": sw["what"]}
+    out["roofline"]["measured_peaks_keys"] = peaks.get("keys")
     if r["e2e"]:
         out["e2e"] = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                       "h2d_bytes_per_step": r["e2e"]["h2d_bytes_per_step"],
@@ -776,6 +1038,8 @@ def main(argv=None):
         out["cpu_baseline"] = {"value": cpu["tflops"], "unit": "TFLOP/s", "cores": cpu["cores"],
                                "kind": "oracle", "sample": cpu["sample"]}
     print(json.dumps(out), flush=True)
+    if r.get("sweep") and not r["sweep"]["lm_head_check"]["ok"]:
+        sys.exit("the LM head output failed its sampled check against the float64 definition")
 
 
 def kernel_source_hash() -> str:

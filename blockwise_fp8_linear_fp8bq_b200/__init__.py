@@ -24,9 +24,10 @@ __all__ = [
     "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
     "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
     "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "rmsnorm_quantize",
+    "quantize_group",
     "Operand",
     "row_operand", "block_operand", "mx_operand", "bf16_operand", "gemm", "gemm_workspace", "linear_forward",
-    "linear_dgrad", "linear_wgrad", "check",
+    "linear_dgrad", "linear_wgrad", "set_clock_counters", "check",
 ]
 
 SCALE_FP32 = 0
@@ -62,6 +63,24 @@ class _COperand(ctypes.Structure):
     ]
 
 
+class _CQuantJob(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("x", ctypes.c_void_p),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+        ("ldx", ctypes.c_int64),
+        ("q", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("qt", ctypes.c_void_p),
+        ("scales_t", ctypes.c_void_p),
+    ]
+
+
+QUANT_KINDS = {"act": 0, "act_t": 1, "dual": 2, "weight": 3}
+
+
 def lib_path() -> str:
     return _LIB_PATH
 
@@ -90,6 +109,8 @@ def lib():
         L.fp8bq_rmsnorm_quantize.argtypes = [vp, i64, i64, i64, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, vp]
         L.fp8bq_quantize_act_dual_mx.restype = i32
         L.fp8bq_quantize_act_dual_mx.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
+        L.fp8bq_quantize_group.restype = i32
+        L.fp8bq_quantize_group.argtypes = [ctypes.POINTER(_CQuantJob), i32, i32, vp]
         L.fp8bq_gemm.restype = i32
         L.fp8bq_gemm.argtypes = [ctypes.POINTER(_COperand), ctypes.POINTER(_COperand), vp, i64, i64,
                                  i64, i64, ctypes.c_uint32, vp]
@@ -104,6 +125,8 @@ def lib():
         L.fp8bq_scales_bytes.argtypes = [i32, i32, i64, i64]
         L.fp8bq_check.restype = i32
         L.fp8bq_check.argtypes = [vp]
+        L.fp8bq_set_clock_counters.restype = i32
+        L.fp8bq_set_clock_counters.argtypes = [vp]
         L.fp8bq_last_cuda_error.restype = i32
         L.fp8bq_status_string.restype = ctypes.c_char_p
         L.fp8bq_status_string.argtypes = [i32]
@@ -290,6 +313,50 @@ def quantize_weight(w: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None):
     return q, s
 
 
+def quantize_group(jobs, fmt: int = SCALE_FP32):
+    """Several quantizations in one launch (fp8bq_quantize_group).  Each job is
+    (kind, x) or (kind, x, outputs) with kind one of "act", "act_t", "dual",
+    "weight"; outputs, when given, are the tensors the single call of that kind
+    would return ((q, s), (qt, st), (q, s, qt, st), (q, s)).  Returns the
+    list of each job's outputs, bit-identical to the single calls'."""
+    if not 1 <= len(jobs) <= 8:
+        raise ValueError("1 to 8 jobs")
+    cjobs = (_CQuantJob * len(jobs))()
+    results = []
+    dev = None
+    for i, job in enumerate(jobs):
+        kind, x = job[0], job[1]
+        given = job[2] if len(job) > 2 else None
+        _check_bf16(x, "x")
+        dev = x.device if dev is None else dev
+        if x.device != dev:
+            raise ValueError("all jobs on one device")
+        M, K = x.shape
+        sdt = _scale_dtype(fmt)
+        e4 = torch.float8_e4m3fn
+        o = list(given) if given is not None else None
+        if kind == "act":
+            outs = (_out(o and o[0], (M, K), e4, dev), _out(o and o[1], (K // 128, row_scale_ld(M)), sdt, dev))
+            q, sc, qt, st = outs[0], outs[1], None, None
+        elif kind == "act_t":
+            outs = (_out(o and o[0], (K, M), e4, dev), _out(o and o[1], (M // 128, row_scale_ld(K)), sdt, dev))
+            q, sc, qt, st = None, None, outs[0], outs[1]
+        elif kind == "dual":
+            outs = (_out(o and o[0], (M, K), e4, dev), _out(o and o[1], (K // 128, row_scale_ld(M)), sdt, dev),
+                    _out(o and o[2], (K, M), e4, dev), _out(o and o[3], (M // 128, row_scale_ld(K)), sdt, dev))
+            q, sc, qt, st = outs
+        elif kind == "weight":
+            outs = (_out(o and o[0], (M, K), e4, dev), _out(o and o[1], (K // 128, (M + 127) // 128), sdt, dev))
+            q, sc, qt, st = outs[0], outs[1], None, None
+        else:
+            raise ValueError(f"unknown job kind {kind!r}")
+        ptr = lambda t: t.data_ptr() if t is not None else None
+        cjobs[i] = _CQuantJob(QUANT_KINDS[kind], 0, x.data_ptr(), M, K, x.stride(0), ptr(q), ptr(sc), ptr(qt), ptr(st))
+        results.append(outs)
+    _raise(lib().fp8bq_quantize_group(cjobs, len(jobs), fmt, _stream(jobs[0][1])), "fp8bq_quantize_group")
+    return results
+
+
 @dataclass
 class Operand:
     """A GEMM operand seen as a logical [rows, C] matrix (C = contraction)."""
@@ -403,6 +470,20 @@ def linear_wgrad(dy: torch.Tensor, x: torch.Tensor, fmt: int = SCALE_FP32) -> to
     qdt, sdt = quantize_act_t(dy, fmt)
     qxt, sxt = quantize_act_t(x, fmt)
     return gemm(row_operand(qdt, sdt, fmt), row_operand(qxt, sxt, fmt))
+
+
+def set_clock_counters(counters: Optional[torch.Tensor]) -> None:
+    """GEMM launches on the current device issued after this call add their
+    CTAs' SM cycles and nanoseconds to counters[0] and counters[1] (a zeroed
+    int64 CUDA tensor of 2 entries); None stops.  counters[0] / counters[1]
+    is the SM clock in GHz the GEMMs ran at."""
+    if counters is None:
+        _raise(lib().fp8bq_set_clock_counters(None), "fp8bq_set_clock_counters")
+        return
+    if not counters.is_cuda or counters.dtype != torch.int64 or counters.numel() < 2 or not counters.is_contiguous():
+        raise ValueError("counters must be a contiguous int64 CUDA tensor of at least 2 entries")
+    with torch.cuda.device(counters.device):
+        _raise(lib().fp8bq_set_clock_counters(counters.data_ptr()), "fp8bq_set_clock_counters")
 
 
 def check(stream: Optional[torch.cuda.Stream] = None) -> None:

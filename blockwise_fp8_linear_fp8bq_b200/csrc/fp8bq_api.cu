@@ -291,8 +291,34 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
   if (K % 128 != 0) return FP8BQ_ERR_SHAPE;
   if (N == 0 || K == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_quant_weight(w, N, K, ldw, q, scales, fmt,
-                                                reinterpret_cast<cudaStream_t>(stream)));
+  const fp8bq::QuantJob job{w, N, K, ldw, q, scales, nullptr, nullptr, true};
+  return cuda_status(fp8bq::launch_quant_group(&job, 1, fmt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int fp8bq_quantize_group(const fp8bq_quant_job* jobs, int njobs, int fmt, fp8bq_stream_t stream) {
+  if (jobs == nullptr || njobs < 1 || njobs > 8) return FP8BQ_ERR_INVALID_ARG;
+  if (!valid_fmt(fmt)) return FP8BQ_ERR_INVALID_ARG;
+  fp8bq::QuantJob jb[8];
+  for (int i = 0; i < njobs; ++i) {
+    const fp8bq_quant_job& j = jobs[i];
+    const bool rows = j.kind == FP8BQ_QUANT_ACT || j.kind == FP8BQ_QUANT_ACT_DUAL || j.kind == FP8BQ_QUANT_WEIGHT;
+    const bool cols = j.kind == FP8BQ_QUANT_ACT_T || j.kind == FP8BQ_QUANT_ACT_DUAL;
+    if (!rows && !cols) return FP8BQ_ERR_INVALID_ARG;
+    int st = FP8BQ_OK;
+    if (rows && (st = check_quant_args(j.x, j.rows, j.cols, j.ldx, j.q, j.scales, fmt)) != FP8BQ_OK) return st;
+    if (cols && (st = check_quant_args(j.x, j.rows, j.cols, j.ldx, j.qt, j.scales_t, fmt)) != FP8BQ_OK) return st;
+    if (rows && j.cols % 128 != 0) return FP8BQ_ERR_SHAPE;
+    if (cols && j.rows % 128 != 0) return FP8BQ_ERR_SHAPE;
+    if (cols && j.cols % 8 != 0) return FP8BQ_ERR_ALIGN;
+    jb[i] = fp8bq::QuantJob{j.x, j.rows, j.cols, j.ldx, rows ? j.q : nullptr, rows ? j.scales : nullptr,
+                            cols ? j.qt : nullptr, cols ? j.scales_t : nullptr, j.kind == FP8BQ_QUANT_WEIGHT};
+  }
+  bool any = false;
+  for (int i = 0; i < njobs; ++i) any = any || (jb[i].rows > 0 && jb[i].cols > 0);
+  if (!any) return FP8BQ_OK;
+  int st = device_ok();
+  if (st != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_quant_group(jb, njobs, fmt, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int fp8bq_gemm(const fp8bq_operand* A, const fp8bq_operand* B, void* D, int64_t M, int64_t N,
@@ -353,6 +379,13 @@ int fp8bq_check(fp8bq_stream_t stream) {
   cudaError_t e = fp8bq::read_and_clear_device_status(reinterpret_cast<cudaStream_t>(stream), &status);
   if (e != cudaSuccess) return cuda_status(e);
   return status != 0 ? FP8BQ_ERR_TIMEOUT : FP8BQ_OK;
+}
+
+int fp8bq_set_clock_counters(unsigned long long* counters) {
+  if (counters != nullptr && (reinterpret_cast<uintptr_t>(counters) & 7u) != 0) return FP8BQ_ERR_ALIGN;
+  int st = device_ok();
+  if (st != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::set_clock_counters(counters));
 }
 
 int fp8bq_last_cuda_error(void) { return t_last_cuda_error; }

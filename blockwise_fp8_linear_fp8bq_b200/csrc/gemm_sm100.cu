@@ -126,7 +126,33 @@ struct Params {
   // that operand's scale bytes are staged and decoded to the FP32 value 2^e.
   int a_u8, b_u8;
   int withhold_cluster;  // test hook: this pair never raises its split flags (-1: none)
+  // Clock counters (nullptr: off): every CTA adds the SM cycles (clock64) and
+  // the nanoseconds (globaltimer) between its start and its end, so that
+  // clk[0] / clk[1] is the SM clock in GHz the GEMM ran at.
+  unsigned long long* clk;
 };
+
+// Start / end stamps of a CTA for Params::clk (thread 0 only).
+struct ClockStamp {
+  long long c0;
+  uint64_t t0;
+};
+__device__ __forceinline__ ClockStamp clock_begin(const Params& p) {
+  ClockStamp st{0, 0};
+  if (p.clk != nullptr && threadIdx.x == 0) {
+    st.c0 = clock64();
+    st.t0 = global_timer_ns();
+  }
+  return st;
+}
+__device__ __forceinline__ void clock_end(const Params& p, const ClockStamp& st) {
+  if (p.clk != nullptr && threadIdx.x == 0) {
+    const long long c1 = clock64();
+    const uint64_t t1 = global_timer_ns();
+    atomicAdd(p.clk, static_cast<unsigned long long>(c1 - st.c0));
+    atomicAdd(p.clk + 1, static_cast<unsigned long long>(t1 - st.t0));
+  }
+}
 
 // FP32 value of a UE8M0 scale byte u (2^(u - 127)); u = 0 is the subnormal
 // 2^-127.  The quantizers write u in [0, 254].
@@ -250,7 +276,7 @@ __device__ __forceinline__ void store_tile(const Params& p, const float2 (&acc)[
 // box waits for the previous store to have read the buffer.
 template <int NBOX>
 __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)[32 * NBOX], uint8_t* stage,
-                                            int lane, int m0, int n0) {
+                                            int lane, int m0, int n0, int jump = 0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
   for (int j = 0; j < NBOX; ++j) {
@@ -268,7 +294,7 @@ __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      const int x = n0 + 64 * j;
+      const int x = n0 + 64 * j + (2 * j >= NBOX ? jump : 0);  // the second half of the boxes starts `jump` later
       if (x < p.N && m0 < p.M) tma_store_2d(&p.tmD, sbase, x, m0);
       bulk_commit_group();
     }
@@ -304,7 +330,7 @@ __device__ __forceinline__ void store_boxes_f32(const CUtensorMap* map, const fl
 // through one 4 KB buffer, each added into global memory by a TMA reduce.
 template <int NBOX>
 __device__ __forceinline__ void add_boxes_f32(const CUtensorMap* map, int xlim, int ylim, const float2 (&acc)[16 * NBOX],
-                                              uint8_t* stage, int lane, int m0, int n0) {
+                                              uint8_t* stage, int lane, int m0, int n0, int jump = 0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
   for (int j = 0; j < NBOX; ++j) {
@@ -318,7 +344,7 @@ __device__ __forceinline__ void add_boxes_f32(const CUtensorMap* map, int xlim, 
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      const int x = n0 + 32 * j;
+      const int x = n0 + 32 * j + (2 * j >= NBOX ? jump : 0);  // the second half of the boxes starts `jump` later
       if (x < xlim && m0 < ylim) tma_reduce_add_2d(map, sbase, x, m0);
       bulk_commit_group();
     }
@@ -369,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const ClockStamp clk0 = clock_begin(p);
   const uint32_t tmem_base = *tmem_holder;
   const int KB = p.num_kb;
 
@@ -640,6 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  clock_end(p, clk0);
 }
 
 // ===================================================== CTA-pair kernel ===
@@ -670,6 +698,10 @@ constexpr int P_BN = 256;    // tile columns
 constexpr int P_BNC = 128;   // B rows loaded per CTA
 constexpr uint32_t P_kTileA = P_BMC * BK;  // 16 KB
 constexpr uint32_t P_kTileB = P_BNC * BK;  // 16 KB
+// Register split of the FP32 promotion variant (setmaxnreg), per thread.
+constexpr uint32_t kCtrlRegs = 40;
+constexpr uint32_t kEpiRegs = 232;
+static_assert(4 * kCtrlRegs + 8 * kEpiRegs <= 12 * 168, "register split within the launch allocation");
 // Output staging is one 4 KB box per epilogue warp (two boxes stored one
 // after the other), which leaves room for five operand stages.  Eight
 // epilogue warps of 128 columns each.  (Sixteen warps of 64 columns, capped
@@ -687,9 +719,9 @@ struct Cfg {
   static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
   static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
   static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
-  // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final;
+  // full, fullsc, empty, sfready, scempty [S]; tfull[4], tempty[4], final;
   // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps)
-  static constexpr uint32_t kNumBars = 5 * kStages + 5 + kEpiWarps;
+  static constexpr uint32_t kNumBars = 5 * kStages + 9 + kEpiWarps;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
@@ -726,10 +758,12 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   auto empty_bar = [&](int s) { return bar(2 * P_STAGES + s); };
   auto sfready_bar = [&](int s) { return bar(3 * P_STAGES + s); };
   auto scempty_bar = [&](int s) { return bar(4 * P_STAGES + s); };
-  auto tfull_bar = [&](int b) { return bar(5 * P_STAGES + b); };
-  auto tempty_bar = [&](int b) { return bar(5 * P_STAGES + 2 + b); };
-  const uint32_t final_bar = bar(5 * P_STAGES + 4);
-  auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 5 + w); };
+  // accumulator buffers: UE8M0 / MX one (0); FP32 four 128-column partial
+  // buffers, q = 2 (K block parity) + column half
+  auto tfull_bar = [&](int q) { return bar(5 * P_STAGES + q); };
+  auto tempty_bar = [&](int q) { return bar(5 * P_STAGES + 4 + q); };
+  const uint32_t final_bar = bar(5 * P_STAGES + 8);
+  auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 9 + w); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
@@ -744,9 +778,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       mbar_init(sfready_bar(s), 1);
       mbar_init(scempty_bar(s), C::kEpiWarps);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 2 * C::kEpiWarps);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(tfull_bar(q), 1);
+      // FP32: a half buffer is drained by the four epilogue warps of its
+      // column half in each CTA; UE8M0: the accumulator by all of them
+      mbar_init(tempty_bar(q), kFp32 ? C::kEpiWarps : 2 * C::kEpiWarps);
     }
     mbar_init(final_bar, 1);
     for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(eload_bar(w), 1);
@@ -760,13 +796,25 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   tc_fence_before();
   cluster_sync();  // barriers of both CTAs initialized, TMEM of both allocated
   tc_fence_after();
+  const ClockStamp clk0 = clock_begin(p);
   const uint32_t tmem_base = *tmem_holder;
   const int cl = static_cast<int>(cluster_id_x());
   const int ncl = static_cast<int>(nclusters_x());
+  // FP32 promotion: the epilogue holds 128 FP32 accumulators and two
+  // 32-column partial chunks per thread, so the control warpgroup (warps
+  // 0-3) hands registers over to the two epilogue warpgroups: 4 warps x 40
+  // plus 8 warps x 232 is exactly the 12 x 168 the CTA was launched with.
+  // Each role sets its budget at its own entry, so the compiler allots each
+  // role's code its own register count (the bounded waits are inlined for
+  // the same reason: an out-of-line callee cannot serve both budgets).
+  auto ctrl_regs = [&]() {
+    if constexpr (kFp32) regs_dealloc<pairk::kCtrlRegs>();
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // Warp-uniform loop; one elected lane issues the copies.
+    ctrl_regs();
     prefetch_tensormap(&p.tmA);
     prefetch_tensormap(&p.tmB);
     if (kMx) {
@@ -837,24 +885,54 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     // ----------------------------------------------------------------- MMA
     // The whole warp runs the loop, so descriptors and TMEM addresses stay
     // warp-uniform; one elected lane issues the tcgen05 instructions.
+    ctrl_regs();
     if (leader) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
+      // FP32: N = 128 per MMA (each half of the 256-column tile committed on
+      // its own); UE8M0 / MX: N = 256
+      const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN / 2, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
       for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
-          uint32_t d = tmem_base;
-          if (kFp32) {
-            const uint32_t b = it & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(b), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) { ok = false; break; }
-            d = tmem_base + b * 256;
-          }
+          const uint32_t d = tmem_base;
           if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kTimeoutMma))) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
           const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
+          if constexpr (kFp32) {
+            // Promotion: K block kb writes a fresh partial into the buffers
+            // 2 (kb parity) + h, h the column half.  MMA h reads rows 64 h ..
+            // 64 h + 63 of each CTA's 128 B rows (both CTAs': N = 128 over
+            // the pair), so partial column c of half h is tile column 64 h + c
+            // (c < 64) or 128 + 64 h + c - 64.  Each half is committed on its
+            // own barrier: the epilogue warps of that half start on it while
+            // the tensor core computes the other one.
+            const uint32_t pb = it & 1;
+            for (int h = 0; h < 2 && ok; ++h) {
+              const int q = 2 * static_cast<int>(pb) + h;
+              if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(q), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              if (elect_one()) {
+                const uint32_t dq = d + pb * 256 + h * 128;
+#pragma unroll
+                for (int k4 = 0; k4 < BK / 32; ++k4) {
+                  const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
+                  const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 8192 * h + 32 * k4, 16, 1024, kLayoutSw128)
+                                                  : smem_desc(sb + 64 * h + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
+                  mma_f8_pair(dq, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
+                }
+                tc_commit_pair(tfull_bar(q), 0x3);
+                if (h == 1) tc_commit_pair(empty_bar(s), 0x3);
+              }
+              __syncwarp();
+            }
+            if (!ok) break;
+          } else {
           const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
           const uint32_t sf_b = sf_a + 8;
           auto issue_sf = [&]() {
@@ -873,15 +951,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
               // (scale-factor IDs: A at bits 29-30, B at bits 4-5)
               const uint32_t idk = kMx ? (idesc | (static_cast<uint32_t>(k4) << 29) | (static_cast<uint32_t>(k4) << 4))
                                        : idesc;
-              if (kFp32)
-                mma_f8_pair(d, adesc, bdesc, idk, k4 > 0 ? 1u : 0u);
-              else
-                mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > u.kb0 || k4 > 0) ? 1u : 0u);
+              mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > u.kb0 || k4 > 0) ? 1u : 0u);
             }
             tc_commit_pair(empty_bar(s), 0x3);
-            if (kFp32) tc_commit_pair(tfull_bar(it & 1), 0x3);
           };
-          if (!kFp32 && kb == u.kb0) {
+          if (kb == u.kb0) {
             // first K block of a tile (or piece): the scale factors (own TMEM columns)
             // are copied while the epilogue still drains the accumulator of
             // the previous tile; the MMAs wait for it
@@ -891,10 +965,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tc_fence_after();
             if (elect_one()) issue_mma();
           } else if (elect_one()) {
-            if (!kFp32) issue_sf();
+            issue_sf();
             issue_mma();
           }
           __syncwarp();
+          }
         }
         if (!ok) break;
         if (!kFp32 && elect_one()) tc_commit_pair(tfull_bar(0), 0x3);
@@ -907,6 +982,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   } else if (warp == 2 || (kMx && warp == 3)) {
     // ------------------------------------------------------- scale staging
     // MX: warp 2 stages A's scale words, warp 3 B's (four bytes each).
+    ctrl_regs();
     const bool stage_a = !kMx || warp == 2;
     const bool stage_b = !kMx || warp == 3;
     uint32_t it = 0;
@@ -1000,6 +1076,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------ epilogue
     // Warp w reads TMEM lanes 32 (w % 4) .. and a slice of kCols columns.
+    if constexpr (kFp32) regs_alloc<pairk::kEpiRegs>();
     constexpr int kCols = C::kCols;
     constexpr int kAcc = kCols / 2;
     const int ew = warp - kEpiWarp0;
@@ -1021,46 +1098,55 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
+          // this warp's partial buffer: K block parity b, column half = slice
           const uint32_t b = it & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(b), (it >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
+          const int q = 2 * static_cast<int>(b) + slice;
+          if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(q), (it >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
           if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(s), ph, guard, kTimeoutEpilogue))) { ok = false; break; }
           tc_fence_after();
           const uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
           const uint32_t cbase = tmem_base + lane_addr + b * 256 + slice * kCols;
           const float2 sa2 = make_float2(sa, sa);
+          // Partial chunk c (32 columns) holds tile columns 64 slice + 32 c
+          // (c < 2) or 128 + 64 slice + 32 (c - 2): chunks 0-1 lie in B's
+          // first 128-row block of the tile, chunks 2-3 in its second.  Two
+          // chunks are in flight: chunk c + 1 loads while chunk c is
+          // promoted, so each load's latency hides behind multiply-adds.
+          static_assert(kCols == 128, "four 32-column chunks per warp");
+          float ra[32], rb[32];
+          float2 f2lo = sa2, f2hi = sa2;
           if (!B_ROW) {
-            // one 128x128 block of B per 128 columns
-            const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[(slice * kCols) >> 7];
-            const float2 f2 = make_float2(f, f);
-#pragma unroll
-            for (int c = 0; c < kCols / 32; ++c) {
-              float r[32];
-              tmem_ld_32x32b_x32f(cbase + 32 * c, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), f2, acc[16 * c + i]);
-            }
-          } else {
-            // per-column B scales: 16-column loads keep the staging small
-            // enough for the 128 accumulators to stay in registers
-            const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + slice * kAcc;
-#pragma unroll
-            for (int c = 0; c < kCols / 16; ++c) {
-              float r[16];
-              tmem_ld_32x32b_x16f(cbase + 16 * c, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                acc[8 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), __fmul2_rn(sa2, sbv[8 * c + i]),
-                                            acc[8 * c + i]);
-            }
+            const float* blk = reinterpret_cast<const float*>(slot + kSlotBlk);
+            const float flo = sa * blk[0], fhi = sa * blk[1];
+            f2lo = make_float2(flo, flo);
+            f2hi = make_float2(fhi, fhi);
           }
+          const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + 32 * slice;
+          auto promote = [&](const float* r, int c) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              // per-column B scales (row groups) or the block's one factor
+              const float2 g = B_ROW ? __fmul2_rn(sa2, sbv[16 * c + (c >= 2 ? 32 : 0) + i]) : (c < 2 ? f2lo : f2hi);
+              acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), g, acc[16 * c + i]);
+            }
+          };
+          tmem_ld_32x32b_x32f(cbase, ra);
+          tmem_wait_ld_regs32(ra);
+          tmem_ld_32x32b_x32f(cbase + 32, rb);
+          promote(ra, 0);
+          tmem_wait_ld_regs32(rb);
+          tmem_ld_32x32b_x32f(cbase + 64, ra);
+          promote(rb, 1);
+          tmem_wait_ld_regs32(ra);
+          tmem_ld_32x32b_x32f(cbase + 96, rb);
+          promote(ra, 2);
+          tmem_wait_ld_regs32(rb);
+          promote(rb, 3);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) {
-            mbar_arrive_cluster(tempty_leader0 + 8 * b);
+            mbar_arrive_cluster(tempty_leader0 + 8 * q);
             mbar_arrive(scempty_bar(s));
           }
         }
@@ -1077,8 +1163,13 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
+      // Tile columns of this warp's accumulators: FP32, 64 slice .. + 63 and
+      // 128 + 64 slice .. + 63 (the half-N partial layout); otherwise the
+      // contiguous 128 slice .. + 127.
+      const int n0 = nb * P_BN + (kFp32 ? 64 : 128) * slice;
+      constexpr int kJump = kFp32 ? 64 : 0;  // added to the columns of the warp's second 64
       if constexpr (ACC) {
-        add_boxes_f32<kCols / 32>(&p.tmD, p.N, p.M, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+        add_boxes_f32<kCols / 32>(&p.tmD, p.N, p.M, acc, stage, lane, m0, n0, kJump);
       } else {
         if (u.split) {
           const int sub = 8 * static_cast<int>(rank) + ew;  // this warp's slice of the tile
@@ -1152,11 +1243,13 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           }
           if (!ok) break;
         }
-        store_boxes<kCols / 64>(p, acc, stage, lane, m0, nb * P_BN + slice * kCols);
+        store_boxes<kCols / 64>(p, acc, stage, lane, m0, n0, kJump);
       }
     }
     if (lane == 0) bulk_wait_group0();
     __syncwarp();
+  } else {
+    ctrl_regs();  // the idle warp 3 releases its registers with its warpgroup
   }
 
   tc_fence_before();
@@ -1166,6 +1259,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+  clock_end(p, clk0);
 }
 
 // ================================================ fused quantize-on-load ===
@@ -1297,6 +1391,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
   tc_fence_before();
   cluster_sync();
   tc_fence_after();
+  const ClockStamp clk0 = clock_begin(p);
   const uint32_t tmem_base = *tmem_holder;
   const int KB = p.num_kb;
   const int cl = static_cast<int>(cluster_id_x());
@@ -1584,6 +1679,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, kTmemCols);
   }
+  clock_end(p, clk0);
 }
 
 // ------------------------------------------------------------------- host --
@@ -1591,6 +1687,7 @@ __device__ int g_device_status;
 
 struct DeviceInfo {
   unsigned long long ctx = 0;  // context the cached addresses and attributes belong to
+  unsigned long long* clk = nullptr;  // clock counters of later launches (fp8bq_set_clock_counters)
   int sms = 0;
   int* status = nullptr;
   bool attr_set[8] = {};
@@ -1902,6 +1999,7 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.a_u8 = pr.a_u8 ? 1 : 0;
   prm.b_u8 = pr.b_u8 ? 1 : 0;
   prm.withhold_cluster = pr.withhold_cluster;
+  prm.clk = di->clk;
   const int grid = prm.num_tiles < di->sms ? prm.num_tiles : di->sms;
 
   const bool fp32 = pr.fmt == kFmtFp32;
@@ -1950,6 +2048,15 @@ cudaError_t device_sm_count(int* sms) {
   cudaError_t e = device_info(&di);
   if (e != cudaSuccess) return e;
   *sms = di->sms;
+  return cudaSuccess;
+}
+
+cudaError_t set_clock_counters(unsigned long long* counters) {
+  DeviceInfo* di = nullptr;
+  cudaError_t e = device_info(&di);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(g_mu);
+  di->clk = counters;
   return cudaSuccess;
 }
 

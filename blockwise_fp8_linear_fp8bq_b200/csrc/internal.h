@@ -24,13 +24,26 @@ unsigned long long current_context_id();
 
 inline int64_t round_up128(int64_t r) { return (r + 127) / 128 * 128; }
 
-cudaError_t launch_quant_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q,
-                                void* scales, int fmt, cudaStream_t stream);
 // TMA-fed activation quantizer: row-group codes (q != nullptr), token-group
 // codes (qt != nullptr), or both from one read of X; groups of `group` = 128
 // or (UE8M0 only) 32 values.
 cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, void* q, void* s_rows,
                                void* qt, void* s_cols, int fmt, int group, cudaStream_t stream);
+
+// One job of a grouped quantization launch: an activation X [rows, cols]
+// quantized in row groups (q), token groups (qt) or both, or (block) a weight
+// W [rows, cols] in 128x128 blocks (q, s_rows = scales [cols/128][ceil(rows/128)]).
+struct QuantJob {
+  const void* x;
+  int64_t rows, cols, ldx;
+  void* q;
+  void* s_rows;
+  void* qt;
+  void* s_cols;
+  bool block;
+};
+// Up to 8 jobs in one persistent launch (one format, groups of 128).
+cudaError_t launch_quant_group(const QuantJob* jobs, int njobs, int fmt, cudaStream_t stream);
 
 // SwiGLU of [gate | up] fused with the quantization of its output h
 // (row groups, and token groups when qt != nullptr); h optionally stored.
@@ -94,6 +107,11 @@ constexpr int64_t kWsSlotBytes = kWsTileBytes + 16 * 4;
 // Launches the GEMM; returns a cudaError_t (cudaSuccess on success).  Sets
 // *unsupported when the operand combination is not built.
 cudaError_t launch_gemm(const GemmProblem& p, cudaStream_t stream, bool* unsupported);
+
+// GEMM launches on the current device (in its current context) issued after
+// this call add their CTAs' SM cycles and nanoseconds to counters[0..1]
+// (nullptr: stop).
+cudaError_t set_clock_counters(unsigned long long* counters);
 
 // Device status word of the GEMM kernels (0 = ok, else a timeout code).
 // Reads and clears it after synchronizing `stream`.

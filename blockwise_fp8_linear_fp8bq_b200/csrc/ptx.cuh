@@ -56,7 +56,7 @@ struct WaitGuard {
   uint64_t limit_ns;
 };
 
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitGuard& g,
+static __device__ __forceinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, const WaitGuard& g,
                                             int code) {
   const uint64_t start = global_timer_ns();
   for (uint32_t i = 0;; ++i) {
@@ -89,7 +89,7 @@ __device__ __forceinline__ void st_release_gpu(int* p, int v) {
 }
 // Bounded wait for *flag == want (acquire), with the mbarrier waits' timeout
 // and abort rules.
-static __device__ __noinline__ bool flag_wait(const int* flag, int want, const WaitGuard& g, int code) {
+static __device__ __forceinline__ bool flag_wait(const int* flag, int want, const WaitGuard& g, int code) {
   const uint64_t start = global_timer_ns();
   for (uint32_t i = 0;; ++i) {
     if (ld_acquire_gpu(flag) == want) return true;
@@ -202,6 +202,19 @@ __device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t sd
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// The same wait, naming the 32 registers of the load it completes as operands
+// it may modify: no use of them can then be scheduled before it, even when
+// other work (on registers loaded earlier) sits between the load and here.
+__device__ __forceinline__ void tmem_wait_ld_regs32(float* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]), "+f"(r[6]), "+f"(r[7]),
+                 "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]), "+f"(r[12]), "+f"(r[13]), "+f"(r[14]),
+                 "+f"(r[15]), "+f"(r[16]), "+f"(r[17]), "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]),
+                 "+f"(r[22]), "+f"(r[23]), "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]),
+                 "+f"(r[29]), "+f"(r[30]), "+f"(r[31])
+               :
+               : "memory");
 }
 // Each of the warp's 32 threads reads 32 consecutive 32-bit columns of its own
 // TMEM lane (lane = 32 * (warp % 4) + laneid).
@@ -390,7 +403,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return ok != 0;
 }
-static __device__ __noinline__ bool mbar_wait_cluster_slow(uint32_t bar, uint32_t parity, const WaitGuard& g,
+static __device__ __forceinline__ bool mbar_wait_cluster_slow(uint32_t bar, uint32_t parity, const WaitGuard& g,
                                                     int code) {
   const uint64_t start = global_timer_ns();
   for (uint32_t i = 0;; ++i) {

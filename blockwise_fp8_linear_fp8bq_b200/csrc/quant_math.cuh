@@ -62,21 +62,19 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
     g.mul = 0.0f;
     g.byte = 0;
   } else {
-    // From the IEEE fields of amax = 1.f * 2^E:  448 = 1.75 * 2^8, so
-    // amax <= 448 * 2^(E-8) exactly when the significand is <= 1.75
-    // (fraction field <= 0x600000); otherwise one more power is needed.
-    // Subnormal amax lies far below 448 * 2^-127 and takes the clamp.
+    // From the IEEE fields of amax = 1.f * 2^E (amax >= 0, finite):  448 =
+    // 1.75 * 2^8, so amax <= 448 * 2^(E-8) exactly when the significand is
+    // <= 1.75 (fraction field <= 0x600000); otherwise one more power is
+    // needed.  Adding 0x1FFFFF to the bits carries into the exponent field
+    // exactly when the fraction exceeds 0x600000, so the biased result
+    // e + 127 = E + 127 - 8 + carry is one add and one shift.  Subnormal (or
+    // tiny) amax lies below 448 * 2^-127: the clamp at 0 gives e = -127.
+    // e never exceeds 120 for finite amax, so no upper clamp is needed.
     const uint32_t u = __float_as_uint(amax);
-    const int ef = static_cast<int>((u >> 23) & 0xFF);
-    int e;
-    if (amax == 0.0f) {
-      e = 0;
-    } else if (ef == 0) {
-      e = -127;
-    } else {
-      e = (ef - 127) - 8 + (((u & 0x7FFFFFu) > 0x600000u) ? 1 : 0);
-      e = e < -127 ? -127 : (e > 127 ? 127 : e);
-    }
+    int biased = static_cast<int>((u + 0x1FFFFFu) >> 23) - 8;
+    biased = biased < 0 ? 0 : biased;
+    if (amax == 0.0f) biased = 127;
+    const int e = biased - 127;
     g.s = 0.0f;
     g.r = 0.0f;
     g.mul = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);  // 2^-e, normal for e in [-127,127)
@@ -98,43 +96,42 @@ __device__ __forceinline__ GroupScale make_scale(float amax) {
 // sign of a zero input.  Groups with s < 2^-125 (r = 0) set `slow`; the
 // caller then recomputes with the IEEE division (quant8_exact).
 template <int FMT>
-__device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g, bool& slow) {
-  float x[8];
-  x[0] = bf16_lo(v.x); x[1] = bf16_hi(v.x); x[2] = bf16_lo(v.y); x[3] = bf16_hi(v.y);
-  x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
-  uint2 r;
+__device__ __forceinline__ uint32_t quant2_fast(float2 xx, const GroupScale& g) {
   if constexpr (FMT == kFmtFp32) {
     const float2 r2 = make_float2(g.r, g.r);
     const float2 nr2 = make_float2(-g.r, -g.r);
     const float2 s2 = make_float2(g.s, g.s);
-    uint32_t c[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 xx = make_float2(x[2 * k], x[2 * k + 1]);
-      const float2 nx = make_float2(-x[2 * k], -x[2 * k + 1]);
-      float2 y = __fmul2_rn(xx, r2);
-      float2 e = __ffma2_rn(s2, y, nx);
-      y = __ffma2_rn(nr2, e, y);
-      e = __ffma2_rn(s2, y, nx);
-      y = __ffma2_rn(nr2, e, y);
-      c[k] = cvt_e4m3x2(y.x, y.y);
-    }
-    r.x = c[0] | (c[1] << 16);
-    r.y = c[2] | (c[3] << 16);
-    slow |= (g.r == 0.0f);
+    const float2 nx = make_float2(-xx.x, -xx.y);
+    float2 y = __fmul2_rn(xx, r2);
+    float2 e = __ffma2_rn(s2, y, nx);
+    y = __ffma2_rn(nr2, e, y);
+    e = __ffma2_rn(s2, y, nx);
+    y = __ffma2_rn(nr2, e, y);
+    return cvt_e4m3x2(y.x, y.y);
   } else {
     // x * 2^-e is exact (barring underflow to values that encode to zero)
-    const float2 m2 = make_float2(g.mul, g.mul);
-    uint32_t c[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float2 y = __fmul2_rn(make_float2(x[2 * k], x[2 * k + 1]), m2);
-      c[k] = cvt_e4m3x2(y.x, y.y);
-    }
-    r.x = c[0] | (c[1] << 16);
-    r.y = c[2] | (c[3] << 16);
+    const float2 y = __fmul2_rn(xx, make_float2(g.mul, g.mul));
+    return cvt_e4m3x2(y.x, y.y);
   }
-  return r;
+}
+
+// Two values -> two E4M3 codes (low byte: xx.x); see quant2_fast.  A group
+// whose scale is too small for the division-free quotient sets `slow`.
+template <int FMT>
+__device__ __forceinline__ uint32_t quant2_fast(float2 xx, const GroupScale& g, bool& slow) {
+  if constexpr (FMT == kFmtFp32) slow |= (g.r == 0.0f);
+  return quant2_fast<FMT>(xx, g);
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 quant8_fast(const uint4& v, const GroupScale& g, bool& slow) {
+  uint32_t c[4];
+  c[0] = quant2_fast<FMT>(make_float2(bf16_lo(v.x), bf16_hi(v.x)), g);
+  c[1] = quant2_fast<FMT>(make_float2(bf16_lo(v.y), bf16_hi(v.y)), g);
+  c[2] = quant2_fast<FMT>(make_float2(bf16_lo(v.z), bf16_hi(v.z)), g);
+  c[3] = quant2_fast<FMT>(make_float2(bf16_lo(v.w), bf16_hi(v.w)), g);
+  if constexpr (FMT == kFmtFp32) slow |= (g.r == 0.0f);
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
 
 // Eight bf16 -> eight E4M3 codes of fl32(x / s) with the IEEE division.  Kept

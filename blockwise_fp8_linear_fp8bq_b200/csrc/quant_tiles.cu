@@ -43,8 +43,9 @@ struct QCfg {
   static constexpr uint32_t kStage = SW ? 2 * kQStage : kQStage;
   static constexpr uint32_t kOffBar = kStages * kStage;
   static constexpr uint32_t kNumBars = 3 * kStages;  // full[S], empty[S], hready[S]
-  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kSmem = kOffMisc + 16 + 2048;  // + slack for 2048-byte alignment
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // abort flag; then the grouped kernel's
+  static constexpr uint32_t kRedBytes = kStages * kQConsumers * 4;  // per-stage weight-block amax partials
+  static constexpr uint32_t kSmem = kOffMisc + 16 + kRedBytes + 2048;  // + slack for 2048-byte alignment
   static_assert(kSmem <= 232448, "shared memory budget");
 };
 
@@ -227,27 +228,35 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
     s0 = make_scale<FMT>(m0v);
     s1 = make_scale<FMT>(m1v);
   }
-  uint4 wa[2], wb[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    // first column (low halves) and second column (high halves), 8 tokens
-    wa[h] = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x5410), __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x5410),
-                       __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x5410), __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x5410));
-    wb[h] = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x7632), __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x7632),
-                       __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x7632), __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x7632));
-  }
+  // codes straight from the token words: the first column is the low bf16
+  // of each word, the second the high one; two tokens per conversion
   uint2 ca[2], cb[2];
-  bool slow = false;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    ca[h] = quant8_fast<FMT>(wa[h], s0, slow);
-    cb[h] = quant8_fast<FMT>(wb[h], s1, slow);
+    uint32_t c0[4], c1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t lo = w[8 * h + 2 * k], hi = w[8 * h + 2 * k + 1];
+      c0[k] = quant2_fast<FMT>(make_float2(bf16_lo(lo), bf16_lo(hi)), s0);
+      c1[k] = quant2_fast<FMT>(make_float2(bf16_hi(lo), bf16_hi(hi)), s1);
+    }
+    ca[h] = make_uint2(c0[0] | (c0[1] << 16), c0[2] | (c0[3] << 16));
+    cb[h] = make_uint2(c1[0] | (c1[1] << 16), c1[2] | (c1[3] << 16));
   }
-  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, s0.r == 0.0f || s1.r == 0.0f)) {
+    // groups of tiny scale: the IEEE division on the columns split out
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      ca[h] = quant8_exact<FMT>(wa[h], s0);
-      cb[h] = quant8_exact<FMT>(wb[h], s1);
+      const uint4 wa = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x5410),
+                                  __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x5410),
+                                  __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x5410),
+                                  __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x5410));
+      const uint4 wb = make_uint4(__byte_perm(w[8 * h + 0], w[8 * h + 1], 0x7632),
+                                  __byte_perm(w[8 * h + 2], w[8 * h + 3], 0x7632),
+                                  __byte_perm(w[8 * h + 4], w[8 * h + 5], 0x7632),
+                                  __byte_perm(w[8 * h + 6], w[8 * h + 7], 0x7632));
+      ca[h] = quant8_exact<FMT>(wa, s0);
+      cb[h] = quant8_exact<FMT>(wb, s1);
     }
   }
   const uint4 va = xor_bytes(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), j);
@@ -269,6 +278,49 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   } else if (c + 1 < p.lds_k && lead) {
     store_neutral_scale<FMT>(p.s_cols, sidx + 1);
   }
+}
+
+// One 128x128 weight block (the tile itself): the amax over the whole tile
+// (each warp's share as in tile_rows, then the 16 warps' partials through
+// `red` and a named barrier of the consumer warps), one scale, and the codes
+// of the tile's rows.  The block scale lands at (k0/128) * lds_m + m0/128,
+// lds_m being ceil(N/128) for a weight [N, K].
+template <int FMT>
+__device__ __forceinline__ void tile_block(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp, int lane,
+                                           float* red) {
+  const int half = lane >> 4;
+  const int l16 = lane & 15;
+  uint4 v[4];
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[i] = ld_shared_v4(base + tile_chunk(8 * warp + 2 * i + half, l16));
+    m2 = absmax_bf16x2(m2, absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w)));
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+  m2 &= 0x7FFF7FFFu;
+  if (lane == 0) red[warp] = fmaxf(bf16_lo(m2), bf16_hi(m2));
+  named_bar_sync(1, 32 * kQConsumers);
+  float bm = red[0];
+#pragma unroll
+  for (int w = 1; w < kQConsumers; ++w) bm = fmaxf(bm, red[w]);
+  const GroupScale gs = make_scale<FMT>(bm);
+  uint2 c[4];
+  bool slow = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = quant8_fast<FMT>(v[i], gs, slow);
+  if (FMT == kFmtFp32 && __any_sync(0xffffffffu, slow)) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = quant8_exact<FMT>(v[i], gs);
+  }
+  const int64_t r0 = m0 + 8 * warp + half;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t r = r0 + 2 * i;
+    if (r < p.M) *reinterpret_cast<uint2*>(p.q + r * p.K + k0 + 8 * l16) = c[i];
+  }
+  if (warp == 0 && lane == 0) store_scale<FMT>(p.s_rows, (k0 / 128) * p.lds_m + m0 / 128, gs);
 }
 
 template <int FMT, bool ROWS, bool COLS, int G, bool SW, bool NORM>
@@ -416,6 +468,110 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
   }
 }
 
+// ------------------------------------------------------- grouped launch --
+// Several quantizations in one persistent launch: the tiles of job 0, then
+// job 1, ... are one index space that the CTAs stride through, so the small
+// tensors of a layer (a weight and an activation, say) share one pipeline
+// ramp and one tail instead of paying one each.  A job is a row-group,
+// token-group or dual activation quantization, or a 128x128 weight-block one.
+constexpr int kQMaxJobs = 8;
+constexpr int kQModeRows = 1, kQModeCols = 2, kQModeDual = 3, kQModeBlock = 4;
+
+struct QGroup {
+  QParams job[kQMaxJobs];
+  int tile_end[kQMaxJobs];  // exclusive prefix sums of the jobs' tile counts
+  int mode[kQMaxJobs];
+  int njobs;
+  int num_tiles;
+  int* status;
+  uint64_t limit_ns;
+};
+
+__device__ __forceinline__ int job_of(const QGroup& g, int tile, int& local) {
+  int j = 0;
+  while (j + 1 < g.njobs && tile >= g.tile_end[j]) ++j;
+  local = tile - (j > 0 ? g.tile_end[j - 1] : 0);
+  return j;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kQThreads, 1) quant_group_kernel(const __grid_constant__ QGroup g) {
+  using C = QCfg<false>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 2047) &
+                                             ~static_cast<uintptr_t>(2047));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  auto full_bar = [&](int s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](int s) { return smem_u32(&bars[S + s]); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
+  float* red_all = reinterpret_cast<float*>(smem + C::kOffMisc + 16);  // [S][kQConsumers] block partials
+  const WaitGuard guard{abort_flag, g.status, g.limit_ns};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kQConsumers);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kQConsumers) {
+    // ------------------------------------------------------------ producer
+    for (int j = 0; j < g.njobs; ++j) prefetch_tensormap(&g.job[j].tmX);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < g.num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kQTimeoutProducer))) { ok = false; break; }
+      if (elect_one()) {
+        int lt = 0;
+        const QParams& p = g.job[job_of(g, tile, lt)];
+        const int32_t m0 = (lt / p.tiles_k) * 128;
+        const int32_t k0 = (lt % p.tiles_k) * 128;
+        const uint32_t dst = smem_u32(smem + s * C::kStage);
+        // a box wholly past K (ragged K, token groups only) is not loaded
+        const bool second = k0 + 64 < p.K;
+        mbar_arrive_expect_tx(full_bar(s), second ? kQStage : kQBox);
+        tma_load_2d(dst, &p.tmX, full_bar(s), k0, m0);
+        if (second) tma_load_2d(dst + kQBox, &p.tmX, full_bar(s), k0 + 64, m0);
+      }
+      __syncwarp();
+    }
+    const uint32_t total = it;
+    for (uint32_t j = (total > S ? total - S : 0); j < total; ++j)
+      mbar_wait(full_bar(j % S), (j / S) & 1, guard, kQTimeoutProducer);
+  } else {
+    // ------------------------------------------------------------ consumers
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < g.num_tiles; tile += gridDim.x, ++it) {
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kQTimeoutConsumer))) break;
+      int lt = 0;
+      const int j = job_of(g, tile, lt);
+      const QParams& p = g.job[j];
+      const int mode = g.mode[j];
+      const int64_t m0 = static_cast<int64_t>(lt / p.tiles_k) * 128;
+      const int64_t k0 = static_cast<int64_t>(lt % p.tiles_k) * 128;
+      const uint32_t base = smem_u32(smem + s * C::kStage);
+      if (mode == kQModeBlock) {
+        tile_block<FMT>(p, base, m0, k0, warp, lane, red_all + s * kQConsumers);
+      } else {
+        if (mode & kQModeRows) tile_rows<FMT, 128>(p, base, m0, k0, warp, lane);
+        if (mode & kQModeCols) tile_cols<FMT, 128>(p, base, m0, k0, warp, lane);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(s));
+    }
+  }
+}
+
 // 2-D tensor map over bf16 X [rows, cols] (row pitch in bytes); 64 x 128 boxes,
 // 128-byte swizzle; out-of-range elements read as zero.
 bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64_t ldx) {
@@ -439,11 +595,13 @@ cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  static bool attr_set[64] = {};
-  if (!attr_set[dev]) {
+  // the attribute belongs to the context: set again in a new one
+  static unsigned long long attr_ctx[64] = {};
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || attr_ctx[dev] != ctx) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_ctx[dev] = ctx;
   }
   int sms = 0;
   e = device_sm_count(&sms);
@@ -453,7 +611,71 @@ cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <int FMT>
+cudaError_t launch_group(const QGroup& g, cudaStream_t stream) {
+  auto kern = quant_group_kernel<FMT>;
+  constexpr uint32_t kQSmem = QCfg<false>::kSmem;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  static unsigned long long attr_ctx[64] = {};
+  const unsigned long long ctx = current_context_id();
+  if (ctx == 0 || attr_ctx[dev] != ctx) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+    if (e != cudaSuccess) return e;
+    attr_ctx[dev] = ctx;
+  }
+  int sms = 0;
+  e = device_sm_count(&sms);
+  if (e != cudaSuccess) return e;
+  const int grid = g.num_tiles < sms ? g.num_tiles : sms;
+  kern<<<grid, kQThreads, kQSmem, stream>>>(g);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_quant_group(const QuantJob* jobs, int njobs, int fmt, cudaStream_t stream) {
+  if (njobs < 1 || njobs > kQMaxJobs) return cudaErrorInvalidValue;
+  QGroup g;
+  std::memset(&g, 0, sizeof(g));
+  int64_t total = 0;
+  int n = 0;
+  for (int i = 0; i < njobs; ++i) {
+    const QuantJob& jb = jobs[i];
+    if (jb.rows == 0 || jb.cols == 0) continue;
+    QParams& p = g.job[n];
+    if (!encode_x(&p.tmX, jb.x, jb.rows, jb.cols, jb.ldx)) return cudaErrorInvalidValue;
+    p.M = jb.rows;
+    p.K = jb.cols;
+    p.q = static_cast<uint8_t*>(jb.q);
+    p.s_rows = jb.s_rows;
+    p.qt = static_cast<uint8_t*>(jb.qt);
+    p.s_cols = jb.s_cols;
+    p.lds_k = round_up128(jb.cols);
+    p.tiles_k = static_cast<int>((jb.cols + 127) / 128);
+    if (jb.block) {
+      p.lds_m = (jb.rows + 127) / 128;  // weight scales [K/128][ceil(N/128)]
+      g.mode[n] = kQModeBlock;
+    } else {
+      p.lds_m = round_up128(jb.rows);
+      g.mode[n] = (jb.q != nullptr ? kQModeRows : 0) | (jb.qt != nullptr ? kQModeCols : 0);
+      if (g.mode[n] == 0) return cudaErrorInvalidValue;
+    }
+    total += ((jb.rows + 127) / 128) * static_cast<int64_t>(p.tiles_k);
+    if (total > INT32_MAX) return cudaErrorInvalidValue;
+    g.tile_end[n] = static_cast<int>(total);
+    ++n;
+  }
+  if (n == 0) return cudaSuccess;
+  g.njobs = n;
+  g.num_tiles = static_cast<int>(total);
+  cudaError_t e = device_status_word(&g.status);
+  if (e != cudaSuccess) return e;
+  g.limit_ns = 2000000000ull;
+  return fmt == kFmtFp32 ? launch_group<kFmtFp32>(g, stream) : launch_group<kFmtUe8m0>(g, stream);
+}
 
 // X [M, K] -> any of: row-group codes q [M, K] + scales [K/G][round_up(M,128)]
 // (q != nullptr), token-group codes qt [K, M] + scales [M/G][round_up(K,128)]

@@ -247,6 +247,45 @@ int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void
                           int fmt, fp8bq_stream_t stream);
 
 /*
+ * Several quantizations in one launch.  The pages have no such call: it is
+ * the calls above (fp8bq_quantize_act / _act_t / _act_dual /
+ * fp8bq_quantize_weight), run together by one persistent kernel over the
+ * concatenated tiles of all jobs, so that the small tensors of a layer (its
+ * weight and its input, say) share one pipeline ramp and one tail instead of
+ * paying for one each.  Every job's outputs are bit-identical to those of
+ * the single call of its kind on the same arguments.
+ *   kind      FP8BQ_QUANT_ACT (q, scales), FP8BQ_QUANT_ACT_T (qt, scales_t),
+ *             FP8BQ_QUANT_ACT_DUAL (all four), FP8BQ_QUANT_WEIGHT (q, scales
+ *             as fp8bq_quantize_weight: 128x128 blocks of a weight [rows, cols],
+ *             scales [cols/128][ceil(rows/128)]).  Pointers a kind does not use
+ *             are ignored.
+ *   x, rows, cols, ldx   the BF16 input and its shape, as in the single call.
+ *   njobs     1 to 8; fmt, the scale format of every job.  A job with rows
+ *             or cols 0 is skipped.
+ * Errors: those of the single calls, per job (the first failing job's);
+ * ERR_INVALID_ARG for a NULL jobs array, njobs outside 1..8 or an unknown kind.
+ */
+typedef enum {
+  FP8BQ_QUANT_ACT = 0,
+  FP8BQ_QUANT_ACT_T = 1,
+  FP8BQ_QUANT_ACT_DUAL = 2,
+  FP8BQ_QUANT_WEIGHT = 3
+} fp8bq_quant_kind;
+typedef struct fp8bq_quant_job {
+  int32_t kind;
+  int32_t reserved; /* set to 0 */
+  const void* x;
+  int64_t rows;
+  int64_t cols;
+  int64_t ldx;
+  void* q;
+  void* scales;
+  void* qt;
+  void* scales_t;
+} fp8bq_quant_job;
+int fp8bq_quantize_group(const fp8bq_quant_job* jobs, int njobs, int fmt, fp8bq_stream_t stream);
+
+/*
  * Blockwise-FP8 GEMM ("精度" section of the ModelScope post; "方法" of the
  * digest):  D[m, n] = sum over 128-blocks kb of  sA(m,kb) * sB(n,kb) *
  * sum_{k in kb} qA[m,k] * qB[n,k], accumulated in FP32 on the tensor cores,
@@ -360,6 +399,23 @@ int64_t fp8bq_scales_bytes(int gran, int fmt, int64_t rows, int64_t contraction)
  * the stream reported an error.  Clears the recorded state.
  */
 int fp8bq_check(fp8bq_stream_t stream);
+
+/*
+ * Clock counters of the GEMM kernels, for measurement (the pages have no
+ * counterpart).  GEMM launches on the current device issued after this call
+ * add, for each of their CTAs, the SM cycles (clock64) and the nanoseconds
+ * (globaltimer) between the CTA's start and its end to counters[0] and
+ * counters[1]: counters[0] / counters[1] is then the SM clock, in GHz, that
+ * the tensor cores ran at, which the driver's clock readings (sampled every
+ * few milliseconds) do not resolve.  Costs two clock reads and two atomic
+ * adds per CTA.
+ *   counters  DEVICE memory of two uint64 (8-byte aligned), zeroed by the
+ *             caller, or NULL to stop.  Launches already captured into a CUDA
+ *             graph keep the pointer they were captured with.
+ * Errors: ERR_ALIGN (counters not 8-byte aligned), ERR_UNSUPPORTED / ERR_CUDA
+ * (no usable device).
+ */
+int fp8bq_set_clock_counters(unsigned long long* counters);
 
 /* The cudaError_t value behind the last FP8BQ_ERR_CUDA of this thread. */
 int fp8bq_last_cuda_error(void);

@@ -268,3 +268,40 @@ def test_rmsnorm_quantize_argument_checks(L):
     assert g(rstd=P + 2) == ALIGN
     assert g(x=P + 8) == ALIGN
     assert g(M=0) == OK                       # empty: no launch
+
+
+def test_quantize_group_argument_checks(L):
+    import blockwise_fp8_linear_fp8bq_b200 as fp
+    f = L.fp8bq_quantize_group
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
+
+    def job(kind=0, x=P, rows=256, cols=256, ldx=256, q=P, s=P, qt=P, st=P):
+        return fp._CQuantJob(kind, 0, x, rows, cols, ldx, q, s, qt, st)
+
+    def g(*jobs, fmt=0, n=None):
+        arr = (fp._CQuantJob * max(1, len(jobs)))(*jobs)
+        return f(ctypes.addressof(arr), len(jobs) if n is None else n, fmt, None)
+
+    assert f(None, 1, 0, None) == INVALID
+    assert g(job(), n=0) == INVALID
+    assert g(job(), n=9) == INVALID
+    assert g(job(), fmt=2) == INVALID
+    assert g(job(kind=7)) == INVALID
+    assert g(job(q=None)) == INVALID                     # act needs q
+    assert g(job(kind=1, qt=None)) == INVALID            # act_t needs qt
+    assert g(job(kind=3, cols=200, ldx=200)) == SHAPE    # weight: contraction % 128
+    assert g(job(kind=1, rows=200)) == SHAPE             # act_t: tokens % 128
+    assert g(job(kind=2, cols=200, ldx=200)) == SHAPE    # dual: both % 128
+    assert g(job(x=P + 8)) == ALIGN
+    assert g(job(), job(kind=3, s=P + 4)) == ALIGN       # the second job's error
+    assert g(job(rows=0), job(kind=3, cols=0)) == OK     # empty jobs: nothing launched
+    assert g(job(), job(kind=3)) in (CUDA, UNSUPPORTED)  # valid: no device here
+
+
+def test_set_clock_counters_argument_checks(L):
+    f = L.fp8bq_set_clock_counters
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p]
+    assert f(P + 4) == ALIGN
+    assert f(P) in (CUDA, UNSUPPORTED)  # no device here
