@@ -1142,13 +1142,14 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           tmem_ld_32x32b_x32f(cbase + 96, rb);
           promote(ra, 2);
           tmem_wait_ld_regs32(rb);
-          promote(rb, 3);
+          // every load of the buffer has completed: hand it back to the MMA
+          // before the last chunk's multiply-adds
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive_cluster(tempty_leader0 + 8 * q);
-            mbar_arrive(scempty_bar(s));
-          }
+          if (lane == 0) mbar_arrive_cluster(tempty_leader0 + 8 * q);
+          promote(rb, 3);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(scempty_bar(s));  // the scale slot's last read (per-column scales) is done
         }
         if (!ok) break;
       } else {
