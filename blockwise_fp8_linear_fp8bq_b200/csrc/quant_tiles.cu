@@ -113,16 +113,25 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   const int l16 = lane & 15;
   uint4 v[4];
   float m[4];
+  uint32_t p2[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = 8 * warp + 2 * i + half;
     v[i] = ld_shared_v4(base + tile_chunk(r, l16));
-    // packed |max| of the 8 values, reduced over the G / 8 lanes of the group
-    uint32_t m2 = absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w));
+    // packed |max| of the 8 values (even columns in the low half, odd ones in the high)
+    p2[i] = absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w));
+  }
+  // two rows per word (row 2j in the low half, 2j + 1 in the high one), so
+  // one shuffle tree over the G / 8 lanes of the groups serves both rows
 #pragma unroll
-    for (int o = G / 16; o >= 1; o >>= 1) m2 = absmax_bf16x2(m2, __shfl_xor_sync(0xffffffffu, m2, o));
-    m2 &= 0x7FFF7FFFu;
-    m[i] = fmaxf(bf16_lo(m2), bf16_hi(m2));
+  for (int j = 0; j < 2; ++j) {
+    uint32_t w = absmax_bf16x2(__byte_perm(p2[2 * j], p2[2 * j + 1], 0x5410),
+                               __byte_perm(p2[2 * j], p2[2 * j + 1], 0x7632));
+#pragma unroll
+    for (int o = G / 16; o >= 1; o >>= 1) w = absmax_bf16x2(w, __shfl_xor_sync(0xffffffffu, w, o));
+    w &= 0x7FFF7FFFu;
+    m[2 * j] = bf16_lo(w);
+    m[2 * j + 1] = bf16_hi(w);
   }
   GroupScale gs[4];
   if constexpr (FMT == kFmtFp32 && G == 128) {
@@ -199,8 +208,15 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   const uint32_t lbase = (base + box * kQBox + 4 * a + 2048u * jj) ^ ((jj << 7) | (jj << 4)) ^
                          (static_cast<uint32_t>(chunk) << 4);
   uint32_t w[16];  // w[i]: token 16 j + (i ^ j)
+  // bit 10 of lbase is clear (the stage is 2048-byte aligned and the other
+  // terms sit in bits 2-9 and 11 up), so for loads 8-15 the XOR with 1024 is
+  // an addition the load's immediate offset absorbs
 #pragma unroll
-  for (int i = 0; i < 16; ++i) w[i] = ld_shared_u32(lbase ^ static_cast<uint32_t>((i << 7) | ((i & 7) << 4)));
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t a = lbase ^ static_cast<uint32_t>((i << 7) | (i << 4));
+    w[i] = ld_shared_u32(a);
+    w[i + 8] = ld_shared_u32(a + 1024u);
+  }
   // packed |max| over the 16 tokens (both columns at once), then over the
   // 8 lanes of the pair
   uint32_t m2 = 0;
