@@ -126,6 +126,10 @@ struct Params {
   // that operand's scale bytes are staged and decoded to the FP32 value 2^e.
   int a_u8, b_u8;
   int withhold_cluster;  // test hook: this pair never raises its split flags (-1: none)
+  // L2 eviction priority of the operand loads and the output stores
+  // (kHint* bits): an operand streamed through once, and the output, go
+  // first, so that an operand read by the tiles of several waves stays.
+  uint32_t l2_hints;
   // Clock counters (nullptr: off): every CTA adds the SM cycles (clock64) and
   // the nanoseconds (globaltimer) between its start and its end, so that
   // clk[0] / clk[1] is the SM clock in GHz the GEMM ran at.
@@ -153,6 +157,8 @@ __device__ __forceinline__ void clock_end(const Params& p, const ClockStamp& st)
     atomicAdd(p.clk + 1, static_cast<unsigned long long>(t1 - st.t0));
   }
 }
+
+constexpr uint32_t kHintAFirst = 1, kHintBFirst = 2, kHintDFirst = 4;
 
 // FP32 value of a UE8M0 scale byte u (2^(u - 127)); u = 0 is the subnormal
 // 2^-127.  The quantizers write u in [0, 254].
@@ -295,7 +301,12 @@ __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)
     __syncwarp();
     if (lane == 0) {
       const int x = n0 + 64 * j + (2 * j >= NBOX ? jump : 0);  // the second half of the boxes starts `jump` later
-      if (x < p.N && m0 < p.M) tma_store_2d(&p.tmD, sbase, x, m0);
+      if (x < p.N && m0 < p.M) {
+        if (p.l2_hints & kHintDFirst)
+          tma_store_2d_hint(&p.tmD, sbase, x, m0, l2_policy_evict_first());
+        else
+          tma_store_2d(&p.tmD, sbase, x, m0);
+      }
       bulk_commit_group();
     }
   }
@@ -817,6 +828,8 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     ctrl_regs();
     prefetch_tensormap(&p.tmA);
     prefetch_tensormap(&p.tmB);
+    const uint64_t pol_a = (p.l2_hints & kHintAFirst) ? l2_policy_evict_first() : 0;
+    const uint64_t pol_b = (p.l2_hints & kHintBFirst) ? l2_policy_evict_first() : 0;
     if (kMx) {
       prefetch_tensormap(&p.tmSA);
       prefetch_tensormap(&p.tmSB);
@@ -852,11 +865,15 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           const uint32_t fb = mapa_shared(full_bar(s), 0);
           const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
           const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
-          tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
-          if (B_KMAJOR)
-            tma_load_2d_pair(sb, &p.tmB, fb, kb * BK, brow);
+          if (pol_a != 0)
+            tma_load_2d_pair_hint(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0), pol_a);
           else
-            tma_load_2d_pair(sb, &p.tmB, fb, brow, kb * BK);
+            tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
+          const int32_t bc0 = B_KMAJOR ? kb * BK : brow, bc1 = B_KMAJOR ? brow : kb * BK;
+          if (pol_b != 0)
+            tma_load_2d_pair_hint(sb, &p.tmB, fb, bc0, bc1, pol_b);
+          else
+            tma_load_2d_pair(sb, &p.tmB, fb, bc0, bc1);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           if (kMx) {
@@ -1690,6 +1707,7 @@ struct DeviceInfo {
   unsigned long long ctx = 0;  // context the cached addresses and attributes belong to
   unsigned long long* clk = nullptr;  // clock counters of later launches (fp8bq_set_clock_counters)
   int sms = 0;
+  int64_t l2_bytes = 0;
   int* status = nullptr;
   bool attr_set[8] = {};
   bool pair_attr_set[12] = {};
@@ -1732,6 +1750,13 @@ cudaError_t device_info(DeviceInfo** out) {
       d.sms = 0;
       return e;
     }
+    int l2 = 0;
+    e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
+    if (e != cudaSuccess) {
+      d.sms = 0;
+      return e;
+    }
+    d.l2_bytes = l2;
     void* sym = nullptr;
     e = cudaGetSymbolAddress(&sym, g_device_status);  // makes the device's context current if none is
     if (e != cudaSuccess) {
@@ -2000,6 +2025,18 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.a_u8 = pr.a_u8 ? 1 : 0;
   prm.b_u8 = pr.b_u8 ? 1 : 0;
   prm.withhold_cluster = pr.withhold_cluster;
+  {
+    // L2 priorities: an operand larger than half the L2 is streamed (each
+    // of its tiles read by the tiles of one wave) and goes first, as does
+    // the output (written once); a smaller operand, re-read by every wave,
+    // keeps the normal priority and so outlasts them
+    const int64_t half_l2 = di->l2_bytes / 2;
+    const int64_t a_bytes = pr.M * pr.K * (pr.a.bf16 ? 2 : 1), b_bytes = pr.N * pr.K;
+    uint32_t h = kHintDFirst;
+    if (a_bytes > half_l2) h |= kHintAFirst;
+    if (b_bytes > half_l2) h |= kHintBFirst;
+    prm.l2_hints = di->l2_bytes > 0 ? h : 0;
+  }
   prm.clk = di->clk;
   const int grid = prm.num_tiles < di->sms ? prm.num_tiles : di->sms;
 
