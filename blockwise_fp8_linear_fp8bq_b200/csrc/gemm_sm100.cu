@@ -282,7 +282,7 @@ __device__ __forceinline__ void store_tile(const Params& p, const float2 (&acc)[
 // box waits for the previous store to have read the buffer.
 template <int NBOX>
 __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)[32 * NBOX], uint8_t* stage,
-                                            int lane, int m0, int n0, int jump = 0) {
+                                            int lane, int m0, int n0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
   for (int j = 0; j < NBOX; ++j) {
@@ -300,7 +300,7 @@ __device__ __forceinline__ void store_boxes(const Params& p, const float2 (&acc)
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      const int x = n0 + 64 * j + (2 * j >= NBOX ? jump : 0);  // the second half of the boxes starts `jump` later
+      const int x = n0 + 64 * j;
       if (x < p.N && m0 < p.M) {
         if (p.l2_hints & kHintDFirst)
           tma_store_2d_hint(&p.tmD, sbase, x, m0, l2_policy_evict_first());
@@ -341,7 +341,7 @@ __device__ __forceinline__ void store_boxes_f32(const CUtensorMap* map, const fl
 // through one 4 KB buffer, each added into global memory by a TMA reduce.
 template <int NBOX>
 __device__ __forceinline__ void add_boxes_f32(const CUtensorMap* map, int xlim, int ylim, const float2 (&acc)[16 * NBOX],
-                                              uint8_t* stage, int lane, int m0, int n0, int jump = 0) {
+                                              uint8_t* stage, int lane, int m0, int n0) {
   const uint32_t sbase = smem_u32(stage);
 #pragma unroll
   for (int j = 0; j < NBOX; ++j) {
@@ -355,7 +355,7 @@ __device__ __forceinline__ void add_boxes_f32(const CUtensorMap* map, int xlim, 
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      const int x = n0 + 32 * j + (2 * j >= NBOX ? jump : 0);  // the second half of the boxes starts `jump` later
+      const int x = n0 + 32 * j;
       if (x < xlim && m0 < ylim) tma_reduce_add_2d(map, sbase, x, m0);
       bulk_commit_group();
     }
@@ -730,9 +730,9 @@ struct Cfg {
   static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
   static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
   static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
-  // full, fullsc, empty, sfready, scempty [S]; tfull[4], tempty[4], final;
+  // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final;
   // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps)
-  static constexpr uint32_t kNumBars = 5 * kStages + 9 + kEpiWarps;
+  static constexpr uint32_t kNumBars = 5 * kStages + 5 + kEpiWarps;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
@@ -769,12 +769,12 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   auto empty_bar = [&](int s) { return bar(2 * P_STAGES + s); };
   auto sfready_bar = [&](int s) { return bar(3 * P_STAGES + s); };
   auto scempty_bar = [&](int s) { return bar(4 * P_STAGES + s); };
-  // accumulator buffers: UE8M0 / MX one (0); FP32 four 128-column partial
-  // buffers, q = 2 (K block parity) + column half
-  auto tfull_bar = [&](int q) { return bar(5 * P_STAGES + q); };
-  auto tempty_bar = [&](int q) { return bar(5 * P_STAGES + 4 + q); };
-  const uint32_t final_bar = bar(5 * P_STAGES + 8);
-  auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 9 + w); };
+  // accumulator buffers: UE8M0 / MX one (0); FP32 two 256-column partial
+  // buffers, one per K-block parity
+  auto tfull_bar = [&](int b) { return bar(5 * P_STAGES + b); };
+  auto tempty_bar = [&](int b) { return bar(5 * P_STAGES + 2 + b); };
+  const uint32_t final_bar = bar(5 * P_STAGES + 4);
+  auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 5 + w); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
@@ -789,11 +789,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       mbar_init(sfready_bar(s), 1);
       mbar_init(scempty_bar(s), C::kEpiWarps);
     }
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(tfull_bar(q), 1);
-      // FP32: a half buffer is drained by the four epilogue warps of its
-      // column half in each CTA; UE8M0: the accumulator by all of them
-      mbar_init(tempty_bar(q), kFp32 ? C::kEpiWarps : 2 * C::kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * C::kEpiWarps);  // every epilogue warp of both CTAs drains it
     }
     mbar_init(final_bar, 1);
     for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(eload_bar(w), 1);
@@ -906,9 +904,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     if (leader) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      // FP32: N = 128 per MMA (each half of the 256-column tile committed on
-      // its own); UE8M0 / MX: N = 256
-      const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN / 2, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
+      const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
       for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
@@ -919,32 +915,29 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           const uint32_t sa = smem_u32(smem + C::kOffA + s * P_kTileA);
           const uint32_t sb = smem_u32(smem + C::kOffB + s * P_kTileB);
           if constexpr (kFp32) {
-            // Promotion: K block kb writes a fresh partial into the buffers
-            // 2 (kb parity) + h, h the column half.  MMA h reads rows 64 h ..
-            // 64 h + 63 of each CTA's 128 B rows (both CTAs': N = 128 over
-            // the pair), so partial column c of half h is tile column 64 h + c
-            // (c < 64) or 128 + 64 h + c - 64.  Each half is committed on its
-            // own barrier: the epilogue warps of that half start on it while
-            // the tensor core computes the other one.
+            // Promotion: K block kb writes a fresh partial (accumulate off at
+            // its first MMA) into the 256-column buffer of its parity, once
+            // the epilogue has drained that buffer's previous partial.  (Two
+            // N = 128 halves per K block, each on its own barrier, were
+            // measured slower: each tcgen05.mma costs the issuing warp tens
+            // of cycles, and eight of them per K block outran the 512
+            // cycles of tensor work.)
             const uint32_t pb = it & 1;
-            for (int h = 0; h < 2 && ok; ++h) {
-              const int q = 2 * static_cast<int>(pb) + h;
-              if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(q), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) {
-                ok = false;
-                break;
-              }
+            if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(pb), ((it >> 1) & 1) ^ 1, guard, kTimeoutMma))) {
+              ok = false;
+            } else {
               tc_fence_after();
               if (elect_one()) {
-                const uint32_t dq = d + pb * 256 + h * 128;
+                const uint32_t dq = d + pb * 256;
 #pragma unroll
                 for (int k4 = 0; k4 < BK / 32; ++k4) {
                   const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
-                  const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 8192 * h + 32 * k4, 16, 1024, kLayoutSw128)
-                                                  : smem_desc(sb + 64 * h + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
+                  const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
+                                                  : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
                   mma_f8_pair(dq, adesc, bdesc, idesc, k4 > 0 ? 1u : 0u);
                 }
-                tc_commit_pair(tfull_bar(q), 0x3);
-                if (h == 1) tc_commit_pair(empty_bar(s), 0x3);
+                tc_commit_pair(empty_bar(s), 0x3);
+                tc_commit_pair(tfull_bar(pb), 0x3);
               }
               __syncwarp();
             }
@@ -1115,9 +1108,8 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
           const int s = it % P_STAGES;
           const uint32_t ph = (it / P_STAGES) & 1;
-          // this warp's partial buffer: K block parity b, column half = slice
-          const uint32_t b = it & 1;
-          const int q = 2 * static_cast<int>(b) + slice;
+          const uint32_t b = it & 1;  // the partial buffer of this K block's parity
+          const int q = static_cast<int>(b);
           if (!__all_sync(0xffffffffu, mbar_wait(tfull_bar(q), (it >> 1) & 1, guard, kTimeoutEpilogue))) { ok = false; break; }
           if (!__all_sync(0xffffffffu, mbar_wait(sfready_bar(s), ph, guard, kTimeoutEpilogue))) { ok = false; break; }
           tc_fence_after();
@@ -1125,26 +1117,23 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           const float sa = reinterpret_cast<const float*>(slot + kSlotRawA)[row_in_tile];
           const uint32_t cbase = tmem_base + lane_addr + b * 256 + slice * kCols;
           const float2 sa2 = make_float2(sa, sa);
-          // Partial chunk c (32 columns) holds tile columns 64 slice + 32 c
-          // (c < 2) or 128 + 64 slice + 32 (c - 2): chunks 0-1 lie in B's
-          // first 128-row block of the tile, chunks 2-3 in its second.  Two
-          // chunks are in flight: chunk c + 1 loads while chunk c is
-          // promoted, so each load's latency hides behind multiply-adds.
+          // The warp's 128 columns are tile columns 128 slice .. + 127, one
+          // 128x128 block of B.  Two 32-column chunks are in flight: chunk
+          // c + 1 loads while chunk c is promoted, so each load's latency
+          // hides behind multiply-adds.
           static_assert(kCols == 128, "four 32-column chunks per warp");
           float ra[32], rb[32];
-          float2 f2lo = sa2, f2hi = sa2;
+          float2 f2 = sa2;
           if (!B_ROW) {
-            const float* blk = reinterpret_cast<const float*>(slot + kSlotBlk);
-            const float flo = sa * blk[0], fhi = sa * blk[1];
-            f2lo = make_float2(flo, flo);
-            f2hi = make_float2(fhi, fhi);
+            const float f = sa * reinterpret_cast<const float*>(slot + kSlotBlk)[slice];
+            f2 = make_float2(f, f);
           }
-          const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + 32 * slice;
+          const float2* sbv = reinterpret_cast<const float2*>(slot + kSlotRawB) + slice * kAcc;
           auto promote = [&](const float* r, int c) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               // per-column B scales (row groups) or the block's one factor
-              const float2 g = B_ROW ? __fmul2_rn(sa2, sbv[16 * c + (c >= 2 ? 32 : 0) + i]) : (c < 2 ? f2lo : f2hi);
+              const float2 g = B_ROW ? __fmul2_rn(sa2, sbv[16 * c + i]) : f2;
               acc[16 * c + i] = __ffma2_rn(make_float2(r[2 * i], r[2 * i + 1]), g, acc[16 * c + i]);
             }
           };
@@ -1181,13 +1170,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
         if (lane == 0) mbar_arrive_cluster(tempty_leader0);
       }
       const int m0 = mb * (2 * P_BMC) + P_BMC * static_cast<int>(rank) + 32 * quarter;
-      // Tile columns of this warp's accumulators: FP32, 64 slice .. + 63 and
-      // 128 + 64 slice .. + 63 (the half-N partial layout); otherwise the
-      // contiguous 128 slice .. + 127.
-      const int n0 = nb * P_BN + (kFp32 ? 64 : 128) * slice;
-      constexpr int kJump = kFp32 ? 64 : 0;  // added to the columns of the warp's second 64
+      const int n0 = nb * P_BN + slice * kCols;  // this warp's tile columns
       if constexpr (ACC) {
-        add_boxes_f32<kCols / 32>(&p.tmD, p.N, p.M, acc, stage, lane, m0, n0, kJump);
+        add_boxes_f32<kCols / 32>(&p.tmD, p.N, p.M, acc, stage, lane, m0, n0);
       } else {
         if (u.split) {
           const int sub = 8 * static_cast<int>(rank) + ew;  // this warp's slice of the tile
@@ -1261,7 +1246,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           }
           if (!ok) break;
         }
-        store_boxes<kCols / 64>(p, acc, stage, lane, m0, n0, kJump);
+        store_boxes<kCols / 64>(p, acc, stage, lane, m0, n0);
       }
     }
     if (lane == 0) bulk_wait_group0();
