@@ -731,8 +731,9 @@ struct Cfg {
   static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
   static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
   // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final;
-  // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps)
-  static constexpr uint32_t kNumBars = 5 * kStages + 5 + kEpiWarps;
+  // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps);
+  // gfull, gready, gempty [2] (UE8M0 scale-factor groups)
+  static constexpr uint32_t kNumBars = 5 * kStages + 5 + kEpiWarps + 6;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kOffMisc + 16;
   static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
@@ -759,6 +760,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   const int lane = threadIdx.x & 31;
   constexpr bool kFp32 = (FMT == kFmtFp32);
   constexpr bool kMx = (FMT == kFmtMx);  // 1x32 scales: four per 128-long K block
+  // UE8M0 with 1x128 groups or 128x128 blocks: one scale byte per row and K
+  // block, so the four bytes of a tensor-memory scale word hold four K
+  // blocks' scales (a group) and are copied in once per group; each MMA
+  // selects its K block's byte through the scale-factor IDs
+  constexpr bool kPack = (FMT == kFmtUe8m0);
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
 
@@ -775,6 +781,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   auto tempty_bar = [&](int b) { return bar(5 * P_STAGES + 2 + b); };
   const uint32_t final_bar = bar(5 * P_STAGES + 4);
   auto eload_bar = [&](int w) { return bar(5 * P_STAGES + 5 + w); };
+  auto gfull_bar = [&](int g) { return bar(5 * P_STAGES + 5 + C::kEpiWarps + g); };   // a group's raw scales landed
+  auto gready_bar = [&](int g) { return bar(5 * P_STAGES + 7 + C::kEpiWarps + g); };  // its scale words staged (leader)
+  auto gempty_bar = [&](int g) { return bar(5 * P_STAGES + 9 + C::kEpiWarps + g); };  // its copies and MMAs done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   const WaitGuard guard{abort_flag, p.status, p.limit_ns};
@@ -783,7 +792,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     for (int s = 0; s < P_STAGES; ++s) {
       // UE8M0: the scale-staging warps of both CTAs also arrive on full[s]
       // (MX: two staging warps per CTA, one for A's scales, one for B's)
-      mbar_init(full_bar(s), kFp32 ? 1 : (kMx ? 5 : 3));
+      mbar_init(full_bar(s), kMx ? 5 : 1);
       mbar_init(fullsc_bar(s), 1);
       mbar_init(empty_bar(s), 1);
       mbar_init(sfready_bar(s), 1);
@@ -795,6 +804,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     }
     mbar_init(final_bar, 1);
     for (int w = 0; w < C::kEpiWarps; ++w) mbar_init(eload_bar(w), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(gfull_bar(g), 1);
+      mbar_init(gready_bar(g), 2);  // the staging warps of both CTAs
+      mbar_init(gempty_bar(g), 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -828,11 +842,11 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     prefetch_tensormap(&p.tmB);
     const uint64_t pol_a = (p.l2_hints & kHintAFirst) ? l2_policy_evict_first() : 0;
     const uint64_t pol_b = (p.l2_hints & kHintBFirst) ? l2_policy_evict_first() : 0;
-    if (kMx) {
+    if (kMx || kPack) {
       prefetch_tensormap(&p.tmSA);
-      prefetch_tensormap(&p.tmSB);
+      if (kMx || B_ROW) prefetch_tensormap(&p.tmSB);
     }
-    uint32_t it = 0;
+    uint32_t it = 0, gi = 0;
     bool ok = true;
     for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
@@ -856,6 +870,25 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
       for (int kb = u.kb0; kb < u.kb1; ++kb, ++it) {
         const int s = it % P_STAGES;
         const uint32_t ph = (it / P_STAGES) & 1;
+        if (kPack && (kb == u.kb0 || (kb & 3) == 0)) {
+          // a new scale group (K blocks 4g .. 4g + 3): its raw scale bytes,
+          // [4][128] of A and, for row-group B, [4][256] of B, as two boxes
+          // into group slot gi % 2 (the first two stage slots), once the
+          // group that used the slot before is done
+          const int gs = static_cast<int>(gi & 1);
+          if (!__all_sync(0xffffffffu, mbar_wait(gempty_bar(gs), ((gi >> 1) & 1) ^ 1, guard, kTimeoutProducer))) {
+            ok = false;
+            break;
+          }
+          if (elect_one()) {
+            uint8_t* gslot = smem + C::kOffSlot + gs * kSlotBytes;
+            mbar_arrive_expect_tx(gfull_bar(gs), 4u * 128u + (B_ROW ? 4u * 256u : 0u));
+            tma_load_2d(smem_u32(gslot + kSlotRawA), &p.tmSA, gfull_bar(gs), static_cast<int32_t>(row0), kb & ~3);
+            if (B_ROW) tma_load_2d(smem_u32(gslot + kSlotRawB), &p.tmSB, gfull_bar(gs), nb * P_BN, kb & ~3);
+          }
+          __syncwarp();
+          ++gi;
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kTimeoutProducer))) { ok = false; break; }
         if (kFp32 && !__all_sync(0xffffffffu, mbar_wait(scempty_bar(s), ph ^ 1, guard, kTimeoutProducer))) { ok = false; break; }
         if (elect_one()) {
@@ -874,7 +907,9 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tma_load_2d_pair(sb, &p.tmB, fb, bc0, bc1);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
-          if (kMx) {
+          if (kPack) {
+            // the scales travel per group (above)
+          } else if (kMx) {
             // the K block's four 1x32 scale rows of A (128 rows) and of B (256
             // rows) as two 2-D boxes; past-the-end rows read as zeros
             mbar_arrive_expect_tx(fullsc_bar(s), 4u * 128u + 4u * 256u);
@@ -894,15 +929,18 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     const uint32_t total = it;
     for (uint32_t j = (total > P_STAGES ? total - P_STAGES : 0); j < total; ++j) {
       mbar_wait(empty_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
-      mbar_wait(fullsc_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
+      if (!kPack) mbar_wait(fullsc_bar(j % P_STAGES), (j / P_STAGES) & 1, guard, kTimeoutTeardown);
     }
+    // (a group's scale boxes have landed once its MMAs ran: the empty
+    // barriers above come after them)
   } else if (warp == 1) {
     // ----------------------------------------------------------------- MMA
     // The whole warp runs the loop, so descriptors and TMEM addresses stay
     // warp-uniform; one elected lane issues the tcgen05 instructions.
     ctrl_regs();
     if (leader) {
-      uint32_t it = 0, tcount = 0;
+      uint32_t it = 0, tcount = 0, gi = 0;
+      int gs_cur = 0;  // UE8M0: the scale group slot of the K block at hand
       bool ok = true;
       const uint32_t idesc = kFp32 ? idesc_f8(2 * P_BMC, P_BN, !B_KMAJOR) : idesc_mxf8(2 * P_BMC, P_BN, !B_KMAJOR);
       for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
@@ -943,10 +981,21 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             }
             if (!ok) break;
           } else {
-          const uint32_t sf_a = tmem_base + kTmemSf + 16 * s;
+          // scale-factor columns: MX, per stage; UE8M0, per scale group slot
+          const bool group_start = kPack && (kb == u.kb0 || (kb & 3) == 0);
+          if (group_start) {
+            gs_cur = static_cast<int>(gi & 1);
+            if (!__all_sync(0xffffffffu, mbar_wait(gready_bar(gs_cur), (gi >> 1) & 1, guard, kTimeoutMma))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            ++gi;
+          }
+          const uint32_t sf_a = tmem_base + kTmemSf + 16 * (kPack ? gs_cur : s);
           const uint32_t sf_b = sf_a + 8;
           auto issue_sf = [&]() {
-            const uint32_t tm = smem_u32(smem + C::kOffSlot + s * kSlotBytes + kSlotTm);
+            const uint32_t tm = smem_u32(smem + C::kOffSlot + (kPack ? gs_cur : s) * kSlotBytes + kSlotTm);
             tc_cp_32x128b_warpx4_pair(sf_a, smem_desc(tm, 0, 128, kLayoutNone));
             tc_cp_32x128b_warpx4_pair(sf_b, smem_desc(tm + 512, 0, 128, kLayoutNone));
             tc_cp_32x128b_warpx4_pair(sf_b + 4, smem_desc(tm + 1024, 0, 128, kLayoutNone));
@@ -957,14 +1006,19 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
               const uint64_t adesc = smem_desc(sa + 32 * k4, 16, 1024, kLayoutSw128);
               const uint64_t bdesc = B_KMAJOR ? smem_desc(sb + 32 * k4, 16, 1024, kLayoutSw128)
                                               : smem_desc(sb + 4096 * k4, P_kTileB, 1024, kLayoutSw128);
-              // MX: byte k4 of each scale word holds sub-block k4's scale
-              // (scale-factor IDs: A at bits 29-30, B at bits 4-5)
-              const uint32_t idk = kMx ? (idesc | (static_cast<uint32_t>(k4) << 29) | (static_cast<uint32_t>(k4) << 4))
-                                       : idesc;
+              // scale-factor IDs (A at bits 29-30, B at bits 4-5) select the
+              // byte of each scale word: MX, sub-block k4's scale; UE8M0,
+              // K block kb's scale within its group
+              const uint32_t sel = kMx ? static_cast<uint32_t>(k4) : static_cast<uint32_t>(kb & 3);
+              const uint32_t idk = idesc | (sel << 29) | (sel << 4);
               mma_mxf8_pair(d, adesc, bdesc, idk, sf_a, sf_b, (kb > u.kb0 || k4 > 0) ? 1u : 0u);
             }
             tc_commit_pair(empty_bar(s), 0x3);
+            // the group's last K block: its scale words (smem and TMEM) are
+            // free once these MMAs are done
+            if (kPack && ((kb & 3) == 3 || kb == u.kb1 - 1)) tc_commit_pair(gempty_bar(gs_cur), 0x3);
           };
+          const bool copy_sf = !kPack || group_start;
           if (kb == u.kb0) {
             // first K block of a tile (or piece): the scale factors (own TMEM columns)
             // are copied while the epilogue still drains the accumulator of
@@ -975,7 +1029,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
             tc_fence_after();
             if (elect_one()) issue_mma();
           } else if (elect_one()) {
-            issue_sf();
+            if (copy_sf) issue_sf();
             issue_mma();
           }
           __syncwarp();
@@ -995,9 +1049,10 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
     ctrl_regs();
     const bool stage_a = !kMx || warp == 2;
     const bool stage_b = !kMx || warp == 3;
-    uint32_t it = 0;
+    uint32_t it = 0, gi = 0;
     bool ok = true;
     const uint32_t full_leader_base = mapa_shared(full_bar(0), 0);
+    const uint32_t gready_leader_base = mapa_shared(gready_bar(0), 0);
     for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
       tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
@@ -1016,6 +1071,52 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
           cur0 = nxt0;
           cur1 = nxt1;
           load_block_scales(p, nb, kb + 32, sb_fp32, nxt0, nxt1);
+        }
+        if constexpr (kPack) {
+          // UE8M0: the scale words of a group (K blocks 4g .. 4g + 3), byte j
+          // of a row's word the row's scale in K block 4g + j, staged once
+          // per group into its slot when its raw bytes have landed
+          if (kb != u.kb0 && (kb & 3) != 0) continue;
+          const int gs = static_cast<int>(gi & 1);
+          if (!__all_sync(0xffffffffu, mbar_wait(gfull_bar(gs), (gi >> 1) & 1, guard, kTimeoutScale))) {
+            ok = false;
+            break;
+          }
+          ++gi;
+          uint8_t* gslot = smem + C::kOffSlot + gs * kSlotBytes;
+          auto pack4 = [&](const uint8_t* raw, int stride, int i) -> uint32_t {
+            return static_cast<uint32_t>(raw[i]) | (static_cast<uint32_t>(raw[stride + i]) << 8) |
+                   (static_cast<uint32_t>(raw[2 * stride + i]) << 16) | (static_cast<uint32_t>(raw[3 * stride + i]) << 24);
+          };
+          const uint8_t* ra = gslot + kSlotRawA;
+          *reinterpret_cast<uint4*>(gslot + kSlotTm + 16 * lane) =
+              make_uint4(pack4(ra, 128, lane), pack4(ra, 128, 32 + lane), pack4(ra, 128, 64 + lane), pack4(ra, 128, 96 + lane));
+          uint32_t blk[2] = {0, 0};
+          if (!B_ROW) {
+            // the two 128x128 blocks' scales of the group's four K blocks
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int kj = ((kb & ~3) + j) & 31;
+              blk[0] |= (__shfl_sync(0xffffffffu, cur0, kj) & 0xFFu) << (8 * j);
+              blk[1] |= (__shfl_sync(0xffffffffu, cur1, kj) & 0xFFu) << (8 * j);
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 wb;
+            if (B_ROW) {
+              const uint8_t* rb = gslot + kSlotRawB + 128 * h;
+              wb = make_uint4(pack4(rb, 256, lane), pack4(rb, 256, 32 + lane), pack4(rb, 256, 64 + lane),
+                              pack4(rb, 256, 96 + lane));
+            } else {
+              wb = make_uint4(blk[h], blk[h], blk[h], blk[h]);
+            }
+            *reinterpret_cast<uint4*>(gslot + kSlotTm + 512 + 512 * h + 16 * lane) = wb;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(gready_leader_base + 8 * gs);
+          continue;
         }
         if (!__all_sync(0xffffffffu, mbar_wait(fullsc_bar(s), ph, guard, kTimeoutScale))) { ok = false; break; }
         uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
@@ -1974,6 +2075,27 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.sb_stride_k = pr.b.s_stride_k;
   prm.sb_stride_r = pr.b.s_stride_r;
   prm.sb_len = pr.b.row_groups ? pr.b.s_stride_k : 0;
+  if (!mx && pair && !fused && pr.fmt == kFmtUe8m0) {
+    // UE8M0 scales of the CTA-pair kernel travel in groups of four K blocks:
+    // byte matrices [K/128][ld], boxes of 128 (A) or 256 (row-group B) rows
+    // by 4 K blocks; past-the-end rows and K blocks read as zeros
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    const void* sp[2] = {pr.a.scales, pr.b.scales};
+    const int64_t ld[2] = {pr.a.s_stride_k, pr.b.s_stride_k};
+    const uint32_t boxc[2] = {128, 256};
+    CUtensorMap* maps[2] = {&prm.tmSA, &prm.tmSB};
+    for (int i = 0; i < (pr.b.row_groups ? 2 : 1); ++i) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(ld[i]), static_cast<cuuint64_t>(pr.K / 128)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld[i])};
+      cuuint32_t box[2] = {boxc[i], 4};
+      cuuint32_t es[2] = {1, 1};
+      CUresult r = fn(maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(sp[i]), dims, strides, box, es,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+      if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    }
+  }
   if (mx) {
     // 1x32 scale arrays as byte matrices [K/32][ld]; boxes of 4 scale rows
     auto fn = encode_fn();

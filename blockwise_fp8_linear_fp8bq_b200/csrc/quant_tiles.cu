@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
 // ramp and one tail instead of paying one each.  A job is a row-group,
 // token-group or dual activation quantization, or a 128x128 weight-block one.
 constexpr int kQMaxJobs = 8;
-constexpr int kQModeRows = 1, kQModeCols = 2, kQModeDual = 3, kQModeBlock = 4;
+constexpr int kQModeRows = 1, kQModeCols = 2, kQModeBlock = 4;  // rows | cols: both layouts
 
 struct QGroup {
   QParams job[kQMaxJobs];
