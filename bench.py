@@ -50,6 +50,7 @@ METRIC = "blockwise-FP8 GEMM TFLOP/s & % FP8 peak; quantizer GB/s & % HBM (1 B20
 WORKLOAD = ("qwen3-1.7b layer linears (qkv 2048x4096, o 2048x2048, gate_up 2048x12288, "
             "down 6144x2048) fwd+dgrad+wgrad, M=16384 tokens")
 FP8_OVER_BF16 = 2.0  # nominal dense FP8 / BF16 tensor ratio (4.5 / 2.25 PFLOP/s)
+FP8_FLOP_PER_SM_CYCLE = 16384  # dense FP8 tensor-core rate of one SM per clock
 
 
 def linears(M=M_TOKENS):
@@ -996,16 +997,19 @@ def main(argv=None):
                          "ms_per_step": split_ms, "clocks": r["clocks_split"]},
     }
     # the SM clock the GEMM kernels counted themselves (clock64 over
-    # globaltimer, summed over CTAs) during the kernel-split replay; the
-    # roofline against the burst peak scaled to that clock, taking the peak's
-    # own clock as the maximum NVML reports under a burst
+    # globaltimer, summed over CTAs) during the kernel-split replay, and the
+    # tensor cores' own peak at that clock: 16384 dense FP8 FLOP per SM per
+    # cycle (the nominal 4.5 PFLOP/s over 148 SMs; ncu's tensor-pipe activity
+    # times the clock reproduces it on these kernels) x SMs x clock
     kmhz = r.get("gemm_kernel_mhz")
     if kmhz:
-        ref_mhz = peaks.get("sm_mhz") or (r["clocks"] or {}).get("sm_max_mhz") or 1965.0
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        peak_clk = FP8_FLOP_PER_SM_CYCLE * sms * kmhz * 1e6 / 1e12
         out["roofline"]["gemm_kernel_sm_mhz"] = kmhz
-        out["roofline"]["peak_at_kernel_clock"] = fp8_peak * kmhz / ref_mhz
-        out["roofline"]["frac_at_kernel_clock"] = gemm_tflops / (fp8_peak * kmhz / ref_mhz)
-        out["roofline"]["peak_clock_mhz_assumed"] = ref_mhz
+        out["roofline"]["peak_at_kernel_clock"] = peak_clk
+        out["roofline"]["frac_at_kernel_clock"] = gemm_tflops / peak_clk
+        out["roofline"]["peak_at_kernel_clock_note"] = (
+            f"{FP8_FLOP_PER_SM_CYCLE} FP8 FLOP/SM/cycle x {sms} SMs x the clock the GEMM kernels counted")
     if r.get("fp8_ceiling"):
         out["roofline"]["fp8_cublas_8192"] = r["fp8_ceiling"]
     if r.get("fp32"):
