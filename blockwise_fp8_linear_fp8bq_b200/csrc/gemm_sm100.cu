@@ -713,23 +713,28 @@ constexpr uint32_t P_kTileB = P_BNC * BK;  // 16 KB
 constexpr uint32_t kCtrlRegs = 40;
 constexpr uint32_t kEpiRegs = 232;
 static_assert(4 * kCtrlRegs + 8 * kEpiRegs <= 12 * 168, "register split within the launch allocation");
-// Output staging is one 4 KB box per epilogue warp (two boxes stored one
-// after the other), which leaves room for five operand stages.  Eight
-// epilogue warps of 128 columns each.  (Sixteen warps of 64 columns, capped
-// at 96 registers a thread, ran the FP32 promotion slower: it is bound by
-// the FP32 pipe and tensor-memory reads, not by load latency.)
-template <bool FP32>
+// Eight epilogue warps of 128 columns each.  (Sixteen warps of 64 columns,
+// capped at 96 registers a thread, ran the FP32 promotion slower: it is bound
+// by the FP32 pipe and tensor-memory reads, not by load latency.)
+// Each warp stages its output through one 4 KB box (TMA stores, or TMA
+// reduce for FP32 accumulation), which leaves room for five operand stages
+// (measured 5-14% faster than four).  Storing the BF16 rows straight from
+// registers instead, to make room for a sixth stage, ran the UE8M0 GEMMs up
+// to 33% slower: a lane's row is 16 bytes a store, 32 rows apart.
+template <int FMT, bool ACC>
 struct Cfg {
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kCols = 256 / (kEpiWarps / 4);  // accumulator columns per epilogue warp
   static constexpr int kStages = 5;
+  // scale slots: UE8M0, two groups of four K blocks; otherwise one per stage
+  static constexpr int kSlots = (FMT == kFmtUe8m0) ? 2 : kStages;
   static constexpr uint32_t kStage = 4096u;  // one 32 x 64 bf16 output box per warp
   static constexpr uint32_t kOffA = 0;
   static constexpr uint32_t kOffB = kOffA + kStages * P_kTileA;
   static constexpr uint32_t kOffStage = kOffB + kStages * P_kTileB;
   static constexpr uint32_t kOffSlot = kOffStage + kEpiWarps * kStage;
-  static constexpr uint32_t kOffBar = kOffSlot + kStages * kSlotBytes;
+  static constexpr uint32_t kOffBar = kOffSlot + kSlots * kSlotBytes;
   // full, fullsc, empty, sfready, scempty [S]; tfull[2], tempty[2], final;
   // eload[kEpiWarps] (split-tile partial-sum loads of the epilogue warps);
   // gfull, gready, gempty [2] (UE8M0 scale-factor groups)
@@ -739,11 +744,14 @@ struct Cfg {
   static constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
   static_assert(kTmemSf + 16 * kStages <= kTmemCols, "scale-factor columns");
+  // the split-tile head piece stages a warp's 32 x 128 FP32 partial (16 KB)
+  // in the operand stages
+  static_assert(kEpiWarps * 16384u <= kStages * (P_kTileA + P_kTileB), "partial-sum staging");
 };
 }  // namespace pairk
 
 template <int FMT, bool B_KMAJOR, bool B_ROW, bool ACC = false>
-__global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
+__global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ Params p) {
   // ACC: D is FP32 and the tile is added into it (D += A B^T), else BF16 D = A B^T
   using pairk::P_BMC;
@@ -751,7 +759,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1)
   using pairk::P_BNC;
   using pairk::P_kTileA;
   using pairk::P_kTileB;
-  using C = pairk::Cfg<FMT == kFmtFp32>;
+  using C = pairk::Cfg<FMT, ACC>;
   constexpr int P_STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1906,13 +1914,13 @@ bool split_tiles(Params& prm, int C, const GemmProblem& pr) {
 template <int FMT, bool BK_, bool BR_, bool ACC_ = false>
 cudaError_t launch_pair_variant(Params& prm, const GemmProblem& pr, DeviceInfo* di, int slot, cudaStream_t stream) {
   auto kern = gemm_pair_kernel<FMT, BK_, BR_, ACC_>;
-  constexpr uint32_t kSmem = pairk::Cfg<FMT == kFmtFp32>::kSmemAlloc;
+  constexpr uint32_t kSmem = pairk::Cfg<FMT, ACC_>::kSmemAlloc;
   if (!di->pair_attr_set[slot]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t occ = {};
     occ.gridDim = dim3(2 * 148, 1, 1);
-    occ.blockDim = dim3(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1, 1);
+    occ.blockDim = dim3(pairk::Cfg<FMT, ACC_>::kThreads, 1, 1);
     occ.dynamicSmemBytes = kSmem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1932,7 +1940,7 @@ cudaError_t launch_pair_variant(Params& prm, const GemmProblem& pr, DeviceInfo* 
   if (split_tiles(prm, di->pair_clusters[slot], pr)) ncl = di->pair_clusters[slot];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * ncl, 1, 1);
-  cfg.blockDim = dim3(pairk::Cfg<FMT == kFmtFp32>::kThreads, 1, 1);
+  cfg.blockDim = dim3(pairk::Cfg<FMT, ACC_>::kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
