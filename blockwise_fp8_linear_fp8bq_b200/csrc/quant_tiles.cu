@@ -62,6 +62,7 @@ struct QParams {
   void* s_cols;     //       scales [M/128][lds_k]
   int64_t lds_k;
   int tiles_k, num_tiles;
+  uint32_t tk_magic;  // floor((2^32 - 1) / tiles_k): tile index division without a divide
   int* status;
   uint64_t limit_ns;
   // SwiGLU producer: X is h = silu(gate) * up of tmX's [gate | up] columns
@@ -72,6 +73,22 @@ struct QParams {
   const float* rstd;       // [M]
   const uint16_t* gamma;   // BF16 [K]
 };
+
+// Tile t of a job -> (row block, column block) = (t / tiles_k, t % tiles_k):
+// q = floor(t m / 2^32) with m = floor((2^32 - 1) / tiles_k) is the quotient
+// or one less (t < 2^31), so one correction step gives the exact division.
+__device__ __forceinline__ void tile_rc(const QParams& p, int t, int64_t& m0, int64_t& k0) {
+  const uint32_t n = static_cast<uint32_t>(t);
+  const uint32_t d = static_cast<uint32_t>(p.tiles_k);
+  uint32_t q = __umulhi(n, p.tk_magic);
+  uint32_t r = n - q * d;
+  if (r >= d) {
+    ++q;
+    r -= d;
+  }
+  m0 = static_cast<int64_t>(q) * 128;
+  k0 = static_cast<int64_t>(r) * 128;
+}
 
 // h = x * rstd * gamma in fp32 (two roundings), rounded to bf16 (nearest,
 // ties to even): within one bf16 ulp of the exact product.  g is the pair's
@@ -175,13 +192,15 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
   }
 }
 
-// Byte i of r moves to byte i ^ j, for 0 <= j < 8: bytes within each word
-// by j & 3 (one byte permute), then words pairwise when j & 4.
-__device__ __forceinline__ uint4 xor_bytes(const uint4& r, int j) {
-  const uint32_t sel = 0x3210u ^ (static_cast<uint32_t>(j & 3) * 0x1111u);
-  const uint32_t x0 = __byte_perm(r.x, 0, sel), x1 = __byte_perm(r.y, 0, sel);
-  const uint32_t x2 = __byte_perm(r.z, 0, sel), x3 = __byte_perm(r.w, 0, sel);
-  return (j & 4) ? make_uint4(x1, x0, x3, x2) : make_uint4(x0, x1, x2, x3);
+// Byte i of r moves to byte i ^ j, for 0 <= j < 8: one byte permute per
+// output word, taking the bytes of its own word (j < 4) or of its pair
+// partner (j >= 4), each at byte index ^ (j & 3).
+__device__ __forceinline__ uint32_t xor_bytes_selector(int j) {
+  return (0x3210u ^ (static_cast<uint32_t>(j & 3) * 0x1111u)) | ((j & 4) ? 0x4444u : 0u);
+}
+__device__ __forceinline__ uint4 xor_bytes(const uint4& r, uint32_t sel) {
+  return make_uint4(__byte_perm(r.x, r.y, sel), __byte_perm(r.y, r.x, sel), __byte_perm(r.z, r.w, sel),
+                    __byte_perm(r.w, r.z, sel));
 }
 
 // Token groups: warp w takes box w & 1 and its column pairs 4 (w >> 1) ..
@@ -275,8 +294,9 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
       cb[h] = quant8_exact<FMT>(wb, s1);
     }
   }
-  const uint4 va = xor_bytes(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), j);
-  const uint4 vb = xor_bytes(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), j);
+  const uint32_t xsel = xor_bytes_selector(j);
+  const uint4 va = xor_bytes(make_uint4(ca[0].x, ca[0].y, ca[1].x, ca[1].y), xsel);
+  const uint4 vb = xor_bytes(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), xsel);
   const int64_t c = k0 + 64 * box + 2 * (4 * chunk + a);
   const int64_t tok = m0 + 16 * j;
   // the first lane of each token group stores its scale: scales [M/G][lds_k]
@@ -379,8 +399,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       const uint32_t ph = (it / S) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(empty_bar(s), ph ^ 1, guard, kQTimeoutProducer))) { ok = false; break; }
       if (elect_one()) {
-        const int32_t m0 = (tile / p.tiles_k) * 128;
-        const int32_t k0 = (tile % p.tiles_k) * 128;
+        int64_t m0l, k0l;
+        tile_rc(p, tile, m0l, k0l);
+        const int32_t m0 = static_cast<int32_t>(m0l), k0 = static_cast<int32_t>(k0l);
         const uint32_t dst = smem_u32(smem + s * C::kStage);
         if (SW) {
           // gate columns k0 .. k0 + 127 and up columns F + k0 .. (F % 128 == 0)
@@ -413,8 +434,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
     float nrs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     auto norm_load = [&](int tile) {
       if (tile >= p.num_tiles) return;
-      const int64_t tm0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
-      const int64_t tk0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
+      int64_t tm0, tk0;
+      tile_rc(p, tile, tm0, tk0);
       ng = __ldg(reinterpret_cast<const uint4*>(p.gamma + tk0 + 8 * (threadIdx.x % 16)));
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -428,8 +449,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       const int s = it % S;
       const uint32_t ph = (it / S) & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(full_bar(s), ph, guard, kQTimeoutConsumer))) break;
-      const int64_t m0 = static_cast<int64_t>(tile / p.tiles_k) * 128;
-      const int64_t k0 = static_cast<int64_t>(tile % p.tiles_k) * 128;
+      int64_t m0, k0;
+      tile_rc(p, tile, m0, k0);
       const uint32_t base = smem_u32(smem + s * C::kStage);
       if constexpr (SW) {
         // h over the gate tile, in place: thread t takes chunk t % 16 of rows
@@ -548,8 +569,9 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_group_kernel(const __grid_
       if (elect_one()) {
         int lt = 0;
         const QParams& p = g.job[job_of(g, tile, lt)];
-        const int32_t m0 = (lt / p.tiles_k) * 128;
-        const int32_t k0 = (lt % p.tiles_k) * 128;
+        int64_t m0l, k0l;
+        tile_rc(p, lt, m0l, k0l);
+        const int32_t m0 = static_cast<int32_t>(m0l), k0 = static_cast<int32_t>(k0l);
         const uint32_t dst = smem_u32(smem + s * C::kStage);
         // a box wholly past K (ragged K, token groups only) is not loaded
         const bool second = k0 + 64 < p.K;
@@ -573,8 +595,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_group_kernel(const __grid_
       const int j = job_of(g, tile, lt);
       const QParams& p = g.job[j];
       const int mode = g.mode[j];
-      const int64_t m0 = static_cast<int64_t>(lt / p.tiles_k) * 128;
-      const int64_t k0 = static_cast<int64_t>(lt % p.tiles_k) * 128;
+      int64_t m0, k0;
+      tile_rc(p, lt, m0, k0);
       const uint32_t base = smem_u32(smem + s * C::kStage);
       if (mode == kQModeBlock) {
         tile_block<FMT>(p, base, m0, k0, warp, lane, red_all + s * kQConsumers);
@@ -671,6 +693,7 @@ cudaError_t launch_quant_group(const QuantJob* jobs, int njobs, int fmt, cudaStr
     p.s_cols = jb.s_cols;
     p.lds_k = round_up128(jb.cols);
     p.tiles_k = static_cast<int>((jb.cols + 127) / 128);
+    p.tk_magic = p.tiles_k > 0 ? 0xFFFFFFFFu / static_cast<uint32_t>(p.tiles_k) : 0u;
     if (jb.block) {
       p.lds_m = (jb.rows + 127) / 128;  // weight scales [K/128][ceil(N/128)]
       g.mode[n] = kQModeBlock;
@@ -711,6 +734,7 @@ cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx,
   prm.s_cols = s_cols;
   prm.lds_k = round_up128(K);
   prm.tiles_k = static_cast<int>((K + 127) / 128);
+  prm.tk_magic = prm.tiles_k > 0 ? 0xFFFFFFFFu / static_cast<uint32_t>(prm.tiles_k) : 0u;
   const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
   prm.num_tiles = static_cast<int>(tiles);
@@ -755,6 +779,7 @@ cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ld
   prm.s_cols = s_cols;
   prm.lds_k = round_up128(F);
   prm.tiles_k = static_cast<int>(F / 128);
+  prm.tk_magic = prm.tiles_k > 0 ? 0xFFFFFFFFu / static_cast<uint32_t>(prm.tiles_k) : 0u;
   const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
   prm.num_tiles = static_cast<int>(tiles);
@@ -828,6 +853,7 @@ cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ld
   prm.s_cols = s_cols;
   prm.lds_k = round_up128(K);
   prm.tiles_k = static_cast<int>(K / 128);
+  prm.tk_magic = prm.tiles_k > 0 ? 0xFFFFFFFFu / static_cast<uint32_t>(prm.tiles_k) : 0u;
   const int64_t tiles = ((M + 127) / 128) * prm.tiles_k;
   if (tiles > INT32_MAX) return cudaErrorInvalidValue;
   prm.num_tiles = static_cast<int>(tiles);
