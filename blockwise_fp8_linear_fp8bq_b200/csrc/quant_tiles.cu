@@ -124,17 +124,14 @@ __device__ __forceinline__ uint32_t tile_chunk(int r, int c) {
 // Row groups: warp w, half-warp h, lane l16 own rows 8 w + 2 i + h (i < 4),
 // chunk l16 (8 values); the amax is a 16-lane reduction.
 template <int FMT, int G>
-__device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
-                                          int lane) {
+__device__ __forceinline__ void tile_rows_regs(const QParams& p, const uint4 (&v)[4], int64_t m0, int64_t k0,
+                                               int warp, int lane) {
   const int half = lane >> 4;
   const int l16 = lane & 15;
-  uint4 v[4];
   float m[4];
   uint32_t p2[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int r = 8 * warp + 2 * i + half;
-    v[i] = ld_shared_v4(base + tile_chunk(r, l16));
     // packed |max| of the 8 values (even columns in the low half, odd ones in the high)
     p2[i] = absmax_bf16x2(absmax_bf16x2(v[i].x, v[i].y), absmax_bf16x2(v[i].z, v[i].w));
   }
@@ -190,6 +187,17 @@ __device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64
       store_neutral_scale<FMT>(p.s_rows, sg * p.lds_m + r);
     }
   }
+}
+
+// The same, loading the warp's rows (8 warp + 2 i + half, chunk l16) from
+// the staged tile.
+template <int FMT, int G>
+__device__ __forceinline__ void tile_rows(const QParams& p, uint32_t base, int64_t m0, int64_t k0, int warp,
+                                          int lane) {
+  uint4 v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = ld_shared_v4(base + tile_chunk(8 * warp + 2 * i + (lane >> 4), lane & 15));
+  tile_rows_regs<FMT, G>(p, v, m0, k0, warp, lane);
 }
 
 // Byte i of r moves to byte i ^ j, for 0 <= j < 8: one byte permute per
@@ -439,7 +447,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       ng = __ldg(reinterpret_cast<const uint4*>(p.gamma + tk0 + 8 * (threadIdx.x % 16)));
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int64_t r = tm0 + threadIdx.x / 16 + 32 * i;
+        const int64_t r = tm0 + 8 * warp + 2 * i + (lane >> 4);
         nrs[i] = r < p.M ? __ldg(p.rstd + r) : 0.0f;
       }
     };
@@ -452,52 +460,51 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
       int64_t m0, k0;
       tile_rc(p, tile, m0, k0);
       const uint32_t base = smem_u32(smem + s * C::kStage);
-      if constexpr (SW) {
-        // h over the gate tile, in place: thread t takes chunk t % 16 of rows
-        // t / 16 + 32 i (the same swizzled offset in both tiles)
-        const int t = threadIdx.x;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = t / 16 + 32 * i;
-          const uint32_t off = tile_chunk(r, t % 16);
-          const uint4 g = ld_shared_v4(base + off);
-          const uint4 u = ld_shared_v4(base + kQStage + off);
-          const uint4 h = make_uint4(swiglu_bf16x2(g.x, u.x), swiglu_bf16x2(g.y, u.y), swiglu_bf16x2(g.z, u.z),
-                                     swiglu_bf16x2(g.w, u.w));
-          st_shared_v4(base + off, h.x, h.y, h.z, h.w);
-          if (p.h != nullptr && m0 + r < p.M)
-            *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + k0 + 8 * (t % 16)) = h;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(hready_bar(s));
-        if (!__all_sync(0xffffffffu, mbar_wait(hready_bar(s), ph, guard, kQTimeoutConsumer))) break;
-      } else if constexpr (NORM) {
-        // h = x * rstd * gamma over the tile, in place: thread t takes chunk
-        // t % 16 (gamma of those 8 columns) of rows t / 16 + 32 i
-        const int t = threadIdx.x;
-        const int64_t col = k0 + 8 * (t % 16);
-        const float2 g0 = make_float2(bf16_lo(ng.x), bf16_hi(ng.x)), g1 = make_float2(bf16_lo(ng.y), bf16_hi(ng.y));
-        const float2 g2 = make_float2(bf16_lo(ng.z), bf16_hi(ng.z)), g3 = make_float2(bf16_lo(ng.w), bf16_hi(ng.w));
+      // Producer ops (SwiGLU, RMSNorm): warp w computes h for the rows it
+      // quantizes in 1x128 groups (8 w + 2 i + half, chunk l16), stores h in
+      // place of the input tile and quantizes those rows from registers; the
+      // token-group phase, which reads every row, waits for all warps' h.
+      bool rows_done = false;
+      if constexpr (SW || NORM) {
+        const int half = lane >> 4, l16 = lane & 15;
+        uint4 hv[4];
+        float2 g0, g1, g2, g3;
         float rsv[4];
+        if constexpr (NORM) {
+          g0 = make_float2(bf16_lo(ng.x), bf16_hi(ng.x));
+          g1 = make_float2(bf16_lo(ng.y), bf16_hi(ng.y));
+          g2 = make_float2(bf16_lo(ng.z), bf16_hi(ng.z));
+          g3 = make_float2(bf16_lo(ng.w), bf16_hi(ng.w));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) rsv[i] = nrs[i];
-        norm_load(tile + gridDim.x);
+          for (int i = 0; i < 4; ++i) rsv[i] = nrs[i];
+          norm_load(tile + gridDim.x);
+        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int r = t / 16 + 32 * i;
-          const uint32_t off = tile_chunk(r, t % 16);
-          const float2 rs2 = make_float2(rsv[i], rsv[i]);
-          const uint4 x = ld_shared_v4(base + off);
-          const uint4 h = make_uint4(rmsnorm_bf16x2(x.x, rs2, g0), rmsnorm_bf16x2(x.y, rs2, g1),
-                                     rmsnorm_bf16x2(x.z, rs2, g2), rmsnorm_bf16x2(x.w, rs2, g3));
-          st_shared_v4(base + off, h.x, h.y, h.z, h.w);
-          if (p.h != nullptr && m0 + r < p.M) *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + col) = h;
+          const int r = 8 * warp + 2 * i + half;
+          const uint32_t off = tile_chunk(r, l16);
+          if constexpr (SW) {
+            const uint4 g = ld_shared_v4(base + off);
+            const uint4 u = ld_shared_v4(base + kQStage + off);
+            hv[i] = make_uint4(swiglu_bf16x2(g.x, u.x), swiglu_bf16x2(g.y, u.y), swiglu_bf16x2(g.z, u.z),
+                               swiglu_bf16x2(g.w, u.w));
+          } else {
+            const float2 rs2 = make_float2(rsv[i], rsv[i]);
+            const uint4 x = ld_shared_v4(base + off);
+            hv[i] = make_uint4(rmsnorm_bf16x2(x.x, rs2, g0), rmsnorm_bf16x2(x.y, rs2, g1),
+                               rmsnorm_bf16x2(x.z, rs2, g2), rmsnorm_bf16x2(x.w, rs2, g3));
+          }
+          st_shared_v4(base + off, hv[i].x, hv[i].y, hv[i].z, hv[i].w);
+          if (p.h != nullptr && m0 + r < p.M)
+            *reinterpret_cast<uint4*>(p.h + (m0 + r) * p.ldh + k0 + 8 * l16) = hv[i];
         }
+        if (ROWS) tile_rows_regs<FMT, G>(p, hv, m0, k0, warp, lane);
+        rows_done = true;
         __syncwarp();
         if (lane == 0) mbar_arrive(hready_bar(s));
         if (!__all_sync(0xffffffffu, mbar_wait(hready_bar(s), ph, guard, kQTimeoutConsumer))) break;
       }
-      if (ROWS) tile_rows<FMT, G>(p, base, m0, k0, warp, lane);
+      if (ROWS && !rows_done) tile_rows<FMT, G>(p, base, m0, k0, warp, lane);
       if (COLS) tile_cols<FMT, G>(p, base, m0, k0, warp, lane);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(s));
