@@ -57,7 +57,7 @@ constexpr int kEpiWarp0 = 4;
 // one 32-column tensor-memory load.
 constexpr int kEpiWarps = 8;
 constexpr int kTmemCols = 512;
-constexpr int kGroupM = 8;  // M blocks per raster group (L2 reuse of B)
+constexpr int kGroupM = 8;  // M blocks per raster group (L2 reuse of B), unless Params::group_m says otherwise
 
 constexpr uint32_t kTileABytes = BM * BK;  // 16 KB
 constexpr uint32_t kTileBBytes = BN * BK;  // 32 KB
@@ -110,6 +110,7 @@ struct Params {
   int64_t ldd;
   int M, N, K;
   int num_m, num_n, num_tiles, num_kb;
+  int group_m;  // M blocks per raster group: consecutive tiles walk down a group's M blocks, then across N
   int* status;
   uint64_t limit_ns;
   // Split tiles (CTA-pair kernel, BF16 D): tiles [dp_tiles, num_tiles) are
@@ -126,9 +127,9 @@ struct Params {
   // that operand's scale bytes are staged and decoded to the FP32 value 2^e.
   int a_u8, b_u8;
   int withhold_cluster;  // test hook: this pair never raises its split flags (-1: none)
-  // L2 eviction priority of the operand loads and the output stores
-  // (kHint* bits): an operand streamed through once, and the output, go
-  // first, so that an operand read by the tiles of several waves stays.
+  // L2 eviction priority of the A loads and the output stores (kHint*
+  // bits): a streamed A and the output go first, so that operand tiles read
+  // by several tiles stay.
   uint32_t l2_hints;
   // Clock counters (nullptr: off): every CTA adds the SM cycles (clock64) and
   // the nanoseconds (globaltimer) between its start and its end, so that
@@ -158,7 +159,7 @@ __device__ __forceinline__ void clock_end(const Params& p, const ClockStamp& st)
   }
 }
 
-constexpr uint32_t kHintAFirst = 1, kHintBFirst = 2, kHintDFirst = 4;
+constexpr uint32_t kHintAFirst = 1, kHintDFirst = 4;
 
 // FP32 value of a UE8M0 scale byte u (2^(u - 127)); u = 0 is the subnormal
 // 2^-127.  The quantizers write u in [0, 254].
@@ -211,11 +212,11 @@ __device__ __forceinline__ Unit next_unit(const Params& p, const Unit& u, int c,
   return split_unit(p, static_cast<int64_t>(u.tile - p.dp_tiles) * p.num_kb + u.kb1, c, ncl);
 }
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
-  const int group = tile / (kGroupM * num_n);
-  const int first_m = group * kGroupM;
-  const int gsz = min(kGroupM, num_m - first_m);
-  const int r = tile - group * kGroupM * num_n;
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int group = tile / (group_m * num_n);
+  const int first_m = group * group_m;
+  const int gsz = min(group_m, num_m - first_m);
+  const int r = tile - group * group_m * num_n;
   mb = first_m + r % gsz;
   nb = r / gsz;
 }
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
         int mb, nb;
-        tile_coords(tile, p.num_m, p.num_n, mb, nb);
+        tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -528,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
       uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
       if (!B_ROW) {
         load_block_scales(p, nb, 0, kFp32, cur0, cur1);
@@ -598,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_kernel(const __grid_constant
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
       float2 acc[64];
       if (kFp32) {
 #pragma unroll
@@ -849,7 +850,6 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
     prefetch_tensormap(&p.tmA);
     prefetch_tensormap(&p.tmB);
     const uint64_t pol_a = (p.l2_hints & kHintAFirst) ? l2_policy_evict_first() : 0;
-    const uint64_t pol_b = (p.l2_hints & kHintBFirst) ? l2_policy_evict_first() : 0;
     if (kMx || kPack) {
       prefetch_tensormap(&p.tmSA);
       if (kMx || B_ROW) prefetch_tensormap(&p.tmSB);
@@ -858,7 +858,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
     bool ok = true;
     for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
-      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, p.group_m, mb, nb);
       const int64_t row0 = static_cast<int64_t>(mb) * (2 * P_BMC) + P_BMC * rank;  // this CTA's A rows
       const int32_t brow = nb * P_BN + P_BNC * static_cast<int>(rank);
       // scale bytes per entry; a UE8M0 operand of the FP32 path lands as raw
@@ -909,10 +909,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
           else
             tma_load_2d_pair(sa, &p.tmA, fb, kb * BK, static_cast<int32_t>(row0));
           const int32_t bc0 = B_KMAJOR ? kb * BK : brow, bc1 = B_KMAJOR ? brow : kb * BK;
-          if (pol_b != 0)
-            tma_load_2d_pair_hint(sb, &p.tmB, fb, bc0, bc1, pol_b);
-          else
-            tma_load_2d_pair(sb, &p.tmB, fb, bc0, bc1);
+          tma_load_2d_pair(sb, &p.tmB, fb, bc0, bc1);
           // this CTA's scale vectors (its own 128 A rows; all 256 B columns)
           uint8_t* slot = smem + C::kOffSlot + s * kSlotBytes;
           if (kPack) {
@@ -1063,7 +1060,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
     const uint32_t gready_leader_base = mapa_shared(gready_bar(0), 0);
     for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl)) {
       int mb, nb;
-      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, p.group_m, mb, nb);
       uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
       const bool sb_fp32 = kFp32 && !p.b_u8;  // B's block scales stored as FP32
       if (!B_ROW) {
@@ -1209,7 +1206,7 @@ __global__ void __launch_bounds__(pairk::Cfg<FMT, ACC>::kThreads, 1)
     bool ok = true;
     for (Unit u = first_unit(p, cl, ncl); ok && u.tile >= 0; u = next_unit(p, u, cl, ncl), ++tcount) {
       int mb, nb;
-      tile_coords(u.tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(u.tile, p.num_m, p.num_n, p.group_m, mb, nb);
       float2 acc[kAcc];
       if (kFp32) {
 #pragma unroll
@@ -1519,7 +1516,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
       bool ok = true;
       for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
         int mb, nb;
-        tile_coords(tile, p.num_m, p.num_n, mb, nb);
+        tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
         const int32_t row0 = mb * (2 * BMC) + BMC * static_cast<int>(rank);
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
@@ -1622,7 +1619,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
     const uint32_t sfmma_leader_base = mapa_shared(sfmma_bar(0), 0);
     for (int tile = cl; ok && tile < p.num_tiles; tile += ncl) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
       uint32_t cur0 = 0, cur1 = 0, nxt0 = 0, nxt1 = 0;
       if (!B_ROW) {
         load_block_scales(p, nb, 0, kFp32, cur0, cur1);
@@ -1706,7 +1703,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_pair_fused_kernel(const __gr
 
     for (int tile = cl; ok && tile < p.num_tiles; tile += ncl, ++tcount) {
       int mb, nb;
-      tile_coords(tile, p.num_m, p.num_n, mb, nb);
+      tile_coords(tile, p.num_m, p.num_n, p.group_m, mb, nb);
       float2 acc[64];
       const uint32_t it0 = it;
       if (kFp32) {
@@ -2141,15 +2138,25 @@ cudaError_t launch_gemm(const GemmProblem& pr, cudaStream_t stream, bool* unsupp
   prm.b_u8 = pr.b_u8 ? 1 : 0;
   prm.withhold_cluster = pr.withhold_cluster;
   {
-    // L2 priorities: an operand larger than half the L2 is streamed (each
-    // of its tiles read by the tiles of one wave) and goes first, as does
-    // the output (written once); a smaller operand, re-read by every wave,
-    // keeps the normal priority and so outlasts them
+    // L2 priorities: the output (written once) goes first, and so does A
+    // when it is larger than the L2 (streamed: each of its row blocks read
+    // by the tiles of one wave; the gate/up data and weight gradients, A =
+    // dY at 201 MB, run 1-1.5% faster).  A smaller A keeps the normal
+    // priority (marked first, the down projection's forward, A = 100 MB,
+    // ran 3% slower), and so does B even when large: its tiles are read by
+    // every M block of a raster group, and marked first they lost that reuse
+    // to the output stream (LM head forward, B = the 311 MB weight: 4.97 ms
+    // against 4.46 ms unmarked).
     const int64_t half_l2 = di->l2_bytes / 2;
-    const int64_t a_bytes = pr.M * pr.K * (pr.a.bf16 ? 2 : 1), b_bytes = pr.N * pr.K;
+    const int64_t a_bytes = pr.M * pr.K * (pr.a.bf16 ? 2 : 1);
     uint32_t h = kHintDFirst;
-    if (a_bytes > half_l2) h |= kHintAFirst;
-    if (b_bytes > half_l2) h |= kHintBFirst;
+    if (a_bytes > di->l2_bytes) h |= kHintAFirst;
+    // raster: groups of 8 M blocks share each B tile among them; when all of
+    // A fits in half the L2 and B does not (the LM head: 33.5 MB of
+    // activations against a 311 MB weight), one group spans every M block,
+    // so that each B tile is read from HBM once while A stays in L2
+    const int64_t b_bytes = pr.N * pr.K;
+    prm.group_m = (di->l2_bytes > 0 && a_bytes <= half_l2 && b_bytes > half_l2) ? prm.num_m : kGroupM;
     prm.l2_hints = di->l2_bytes > 0 ? h : 0;
   }
   prm.clk = di->clk;
