@@ -37,12 +37,16 @@ def split_plan(M, N, K, slots):
     return (W * C if split else T), T, num_m, num_n
 
 
+GROUP_M = 4  # row blocks per raster group (the kernels' default; these operands all fit in the L2)
+
+
 def tile_rect(t, num_m, num_n):
-    """Output rows/columns of tile t (grouped raster, 8 row blocks a group)."""
-    group = t // (8 * num_n)
-    first = group * 8
-    gsz = min(8, num_m - first)
-    r = t - group * 8 * num_n
+    """Output rows/columns of tile t (grouped raster: consecutive tiles walk
+    down a group's GROUP_M row blocks, then across the columns)."""
+    group = t // (GROUP_M * num_n)
+    first = group * GROUP_M
+    gsz = min(GROUP_M, num_m - first)
+    r = t - group * GROUP_M * num_n
     mb, nb = first + r % gsz, r // gsz
     return slice(256 * mb, 256 * mb + 256), slice(256 * nb, 256 * nb + 256)
 
