@@ -12,7 +12,7 @@
 //         of dY, and the forward + wgrad both layouts of X).
 //
 // A persistent CTA per SM: one producer warp streams 128x128 tiles with TMA
-// (two 64-column boxes, 128-byte swizzle) into a six-stage ring; sixteen
+// (two 64-column boxes, 128-byte swizzle) into a three-stage ring; sixteen
 // consumer warps quantize out of shared memory and store codes and scales
 // straight from registers.  Every wait is bounded (status word, as in the
 // GEMM).
@@ -29,14 +29,18 @@
 namespace fp8bq {
 namespace {
 
-constexpr int kQStages = 6;
+// Three 32 KB stages: measured in one process against 2, 4, 5, 6 and 7, three
+// was the fastest over the layer's launches (the gate/up dY dual pass 136 µs
+// against 150 µs with six; two starved the consumers): a deeper ring only
+// puts more reads in flight against the codes being written.
+constexpr int kQStages = 3;
 constexpr int kQConsumers = 16;                 // consumer warps 0..15; warp 16 produces
 constexpr int kQThreads = 32 * (kQConsumers + 1);
 constexpr uint32_t kQBox = 128 * 128;           // 64 bf16 columns x 128 rows: 16 KB
 constexpr uint32_t kQStage = 2 * kQBox;
 // Shared-memory layout.  SW (SwiGLU producer fused in): a stage holds the
 // gate tile and the up tile (64 KB), three stages, and an h-ready barrier
-// per stage; otherwise one 32 KB tile a stage, six stages.
+// per stage; otherwise one 32 KB tile a stage, kQStages stages.
 template <bool SW>
 struct QCfg {
   static constexpr int kStages = SW ? 3 : kQStages;
