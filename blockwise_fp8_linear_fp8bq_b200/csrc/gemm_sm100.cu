@@ -8,6 +8,12 @@
 // 128x128 weight blocks, MXFP8 on Blackwell) and of the ModelScope post's
 // section "精度：FP8 分块量化与净效率收益" (the linear layers' matmuls in FP8).
 //
+// Two kernels.  gemm_pair_kernel (below; every M > 128, i.e. every shape of
+// the layer) runs CTA pairs (tcgen05 cta_group::2) over 256 x 256 tiles with
+// a 5-stage ring, UE8M0 scales packed four K blocks to a tensor-memory word,
+// a grouped raster and split last rounds.  gemm_kernel, for M <= 128, is the
+// single-CTA form described here.
+//
 // Kernel shape (one CTA per SM, persistent over 128 x 256 output tiles,
 // 12 warps):
 //   warp 0      TMA producer: A and B K-block tiles (128-byte swizzle) and the
