@@ -151,7 +151,9 @@ __device__ __forceinline__ void tile_rows_regs(const QParams& p, const uint4 (&v
     m[2 * j] = bf16_lo(w);
     m[2 * j + 1] = bf16_hi(w);
   }
+  static_assert(FMT == kFmtUe8m0 || G == 128, "FP32 scales come in 1x128 groups");
   GroupScale gs[4];
+  GroupScale own{};  // UE8M0: the scale of row slot l16 mod 4
   if constexpr (FMT == kFmtFp32 && G == 128) {
     // one scale per group, computed by lane 2 i + h and fetched by the others
     float mine = 0.0f;
@@ -164,9 +166,19 @@ __device__ __forceinline__ void tile_rows_regs(const QParams& p, const uint4 (&v
 #pragma unroll
     for (int i = 0; i < 4; ++i) gs[i] = fetch_scale<FMT>(gmine, 2 * i + half);
   } else {
-    // a UE8M0 scale is a few integer operations: cheaper than fetching it
+    // the G / 8 lanes of a group hold the same four row maxima: lane slot i
+    // (i = l16 mod 4) computes row slot i's scale, and every lane fetches the
+    // four multipliers from slots 0..3 of its group (one shuffle each, in
+    // place of three scale computations)
+    const int slot = l16 & 3;
+    const float mine = slot == 0 ? m[0] : slot == 1 ? m[1] : slot == 2 ? m[2] : m[3];
+    own = make_scale<FMT>(mine);
+    const int first = lane & ~(G / 8 - 1);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) gs[i] = make_scale<FMT>(m[i]);
+    for (int i = 0; i < 4; ++i) {
+      gs[i] = own;
+      gs[i].mul = __shfl_sync(0xffffffffu, own.mul, first + i);
+    }
   }
   uint2 c[4];
   bool slow = false;
@@ -178,17 +190,33 @@ __device__ __forceinline__ void tile_rows_regs(const QParams& p, const uint4 (&v
   }
   const int64_t r0 = m0 + 8 * warp + half;
   uint8_t* qrow = p.q + r0 * p.K + k0 + 8 * l16;
-  // the first lane of each group stores its scale: scales [K/G][lds_m]
-  const bool lead = (l16 & (G / 8 - 1)) == 0;
-  const int64_t sg = k0 / G + (l16 * 8) / G;
+  const int64_t sg = k0 / G + (l16 * 8) / G;  // scales [K/G][lds_m]
+  if constexpr (FMT == kFmtFp32) {
+    // the first lane of each group stores its four rows' scales
+    const bool lead = (l16 & (G / 8 - 1)) == 0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int64_t r = r0 + 2 * i;
-    if (r < p.M) {
-      *reinterpret_cast<uint2*>(qrow + 2 * i * p.K) = c[i];
-      if (lead) store_scale<FMT>(p.s_rows, sg * p.lds_m + r, gs[i]);
-    } else if (r < p.lds_m && lead) {
-      store_neutral_scale<FMT>(p.s_rows, sg * p.lds_m + r);
+    for (int i = 0; i < 4; ++i) {
+      const int64_t r = r0 + 2 * i;
+      if (r < p.M) {
+        *reinterpret_cast<uint2*>(qrow + 2 * i * p.K) = c[i];
+        if (lead) store_scale<FMT>(p.s_rows, sg * p.lds_m + r, gs[i]);
+      } else if (r < p.lds_m && lead) {
+        store_neutral_scale<FMT>(p.s_rows, sg * p.lds_m + r);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (r0 + 2 * i < p.M) *reinterpret_cast<uint2*>(qrow + 2 * i * p.K) = c[i];
+    }
+    // lane slot i of each group (i < 4) stores row slot i's scale, its own
+    const int gl = l16 & (G / 8 - 1);
+    if (gl < 4) {
+      const int64_t r = r0 + 2 * gl;
+      if (r < p.M)
+        store_scale<FMT>(p.s_rows, sg * p.lds_m + r, own);
+      else if (r < p.lds_m)
+        store_neutral_scale<FMT>(p.s_rows, sg * p.lds_m + r);
     }
   }
 }
@@ -258,6 +286,7 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   m2 &= 0x7FFF7FFFu;
   const float m0v = bf16_lo(m2), m1v = bf16_hi(m2);
   GroupScale s0, s1;
+  GroupScale own{};  // UE8M0: the scale of column j mod 2 of the pair
   if constexpr (FMT == kFmtFp32 && G == 128) {
     // eight groups per warp: lane 2 a' + b computes column b of pair a'
     float mine = 0.0f;
@@ -272,8 +301,14 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
     s0 = fetch_scale<FMT>(gmine, 2 * a);
     s1 = fetch_scale<FMT>(gmine, 2 * a + 1);
   } else {
-    s0 = make_scale<FMT>(m0v);
-    s1 = make_scale<FMT>(m1v);
+    // the G / 16 lanes of a token group hold the same two column maxima: an
+    // even lane computes the first column's scale, an odd one the second's,
+    // and each lane fetches both multipliers from its lane pair
+    own = make_scale<FMT>((j & 1) ? m1v : m0v);
+    s0 = own;
+    s1 = own;
+    s0.mul = __shfl_sync(0xffffffffu, own.mul, lane & ~1);
+    s1.mul = __shfl_sync(0xffffffffu, own.mul, lane | 1);
   }
   // codes straight from the token words: the first column is the low bf16
   // of each word, the second the high one; two tokens per conversion
@@ -311,20 +346,34 @@ __device__ __forceinline__ void tile_cols(const QParams& p, uint32_t base, int64
   const uint4 vb = xor_bytes(make_uint4(cb[0].x, cb[0].y, cb[1].x, cb[1].y), xsel);
   const int64_t c = k0 + 64 * box + 2 * (4 * chunk + a);
   const int64_t tok = m0 + 16 * j;
-  // the first lane of each token group stores its scale: scales [M/G][lds_k]
-  const bool lead = (j & (G / 16 - 1)) == 0;
-  const int64_t sidx = (m0 / G + (16 * j) / G) * p.lds_k + c;
-  if (c < p.K) {
-    *reinterpret_cast<uint4*>(p.qt + c * p.M + tok) = va;
-    if (lead) store_scale<FMT>(p.s_cols, sidx, s0);
-  } else if (c < p.lds_k && lead) {
-    store_neutral_scale<FMT>(p.s_cols, sidx);
-  }
-  if (c + 1 < p.K) {
-    *reinterpret_cast<uint4*>(p.qt + (c + 1) * p.M + tok) = vb;
-    if (lead) store_scale<FMT>(p.s_cols, sidx + 1, s1);
-  } else if (c + 1 < p.lds_k && lead) {
-    store_neutral_scale<FMT>(p.s_cols, sidx + 1);
+  const int64_t sidx = (m0 / G + (16 * j) / G) * p.lds_k + c;  // scales [M/G][lds_k]
+  if constexpr (FMT == kFmtFp32) {
+    // the first lane of each token group stores its two scales
+    const bool lead = (j & (G / 16 - 1)) == 0;
+    if (c < p.K) {
+      *reinterpret_cast<uint4*>(p.qt + c * p.M + tok) = va;
+      if (lead) store_scale<FMT>(p.s_cols, sidx, s0);
+    } else if (c < p.lds_k && lead) {
+      store_neutral_scale<FMT>(p.s_cols, sidx);
+    }
+    if (c + 1 < p.K) {
+      *reinterpret_cast<uint4*>(p.qt + (c + 1) * p.M + tok) = vb;
+      if (lead) store_scale<FMT>(p.s_cols, sidx + 1, s1);
+    } else if (c + 1 < p.lds_k && lead) {
+      store_neutral_scale<FMT>(p.s_cols, sidx + 1);
+    }
+  } else {
+    if (c < p.K) *reinterpret_cast<uint4*>(p.qt + c * p.M + tok) = va;
+    if (c + 1 < p.K) *reinterpret_cast<uint4*>(p.qt + (c + 1) * p.M + tok) = vb;
+    // the first two lanes of each token group store the scales of the first
+    // and the second column, each its own
+    const int gl = j & (G / 16 - 1);
+    if (gl < 2) {
+      if (c + gl < p.K)
+        store_scale<FMT>(p.s_cols, sidx + gl, own);
+      else if (c + gl < p.lds_k)
+        store_neutral_scale<FMT>(p.s_cols, sidx + gl);
+    }
   }
 }
 
