@@ -802,6 +802,9 @@ def case_launchers(step, fp):
             it["gu"] = torch.randn(M, 2 * K, generator=gen, device=it["x"].device).to(torch.bfloat16)
             out[f"quant_swiglu:{n}"] = ("quant", M * 2 * K * 2 + 2 * M * K + 2 * (K // 128) * M * sb,
                                         lambda it=it: fp.swiglu_quantize(it["gu"], f))
+            # the same with h rounded once from its exact value
+            out[f"quant_swiglu_exact:{n}"] = ("quant", M * 2 * K * 2 + 2 * M * K + 2 * (K // 128) * M * sb,
+                                              lambda it=it: fp.swiglu_quantize(it["gu"], f, exact=True))
         if n in ("qkv", "gate_up"):
             # the projection's input from RMSNorm in one pass: rstd, h = x * rstd * gamma,
             # both code layouts (vs a BF16 h written and read back)

@@ -21,7 +21,8 @@ from typing import Optional
 import torch
 
 __all__ = [
-    "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "Fp8bqError", "lib", "lib_path",
+    "SCALE_FP32", "SCALE_UE8M0", "GRAN_ROW", "GRAN_BLOCK", "GRAN_ROW32", "SWIGLU_EXACT", "Fp8bqError", "lib",
+    "lib_path",
     "row_scale_ld", "quantize_act", "quantize_act_t", "quantize_act_dual", "quantize_weight",
     "quantize_act_mx", "quantize_act_t_mx", "quantize_act_dual_mx", "swiglu_quantize", "rmsnorm_quantize",
     "quantize_group",
@@ -35,6 +36,7 @@ SCALE_UE8M0 = 1
 GRAN_ROW = 0
 GRAN_BLOCK = 1
 GRAN_ROW32 = 2  # MX blocks: 1x32 row groups, UE8M0 scales
+SWIGLU_EXACT = 0x100  # swiglu_quantize: h rounded once from its exact value
 _E4M3 = 0
 _BF16 = 1
 
@@ -221,10 +223,12 @@ def quantize_act_dual(x: torch.Tensor, fmt: int = SCALE_FP32, q=None, s=None, qt
     return q, s, qt, st
 
 
-def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = True, keep_h: bool = False):
+def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = True, keep_h: bool = False,
+                    exact: bool = False):
     """[gate | up] bf16 [M, 2F] -> (q, s, qt, st, h): h = silu(gate) * up in BF16
     quantized as quantize_act (q, s) and, with transposed, quantize_act_t (qt, st);
-    h itself is returned when keep_h (else None), qt/st are None without transposed."""
+    h itself is returned when keep_h (else None), qt/st are None without transposed.
+    exact: h is the exact value rounded once to BF16 (FP8BQ_SWIGLU_EXACT)."""
     _check_bf16(gu, "gu")
     M, F2 = gu.shape
     F = F2 // 2
@@ -235,7 +239,7 @@ def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = 
     h = _out(None, (M, F), torch.bfloat16, gu.device) if keep_h else None
     ptr = lambda t: t.data_ptr() if t is not None else None
     rc = lib().fp8bq_swiglu_quantize(gu.data_ptr(), M, F, gu.stride(0), ptr(h), q.data_ptr(), s.data_ptr(),
-                                     ptr(qt), ptr(st), fmt, _stream(gu))
+                                     ptr(qt), ptr(st), fmt | (SWIGLU_EXACT if exact else 0), _stream(gu))
     _raise(rc, "fp8bq_swiglu_quantize")
     return q, s, qt, st, h
 

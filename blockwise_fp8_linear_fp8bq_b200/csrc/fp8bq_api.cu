@@ -254,6 +254,8 @@ int fp8bq_quantize_act_dual_mx(const void* x, int64_t M, int64_t K, int64_t ldx,
 
 int fp8bq_swiglu_quantize(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* scales,
                           void* qt, void* scales_t, int fmt, fp8bq_stream_t stream) {
+  const bool exact = (fmt & FP8BQ_SWIGLU_EXACT) != 0;
+  fmt &= ~FP8BQ_SWIGLU_EXACT;
   int st = check_quant_args(gu, M, 2 * F, ldgu, q, scales, fmt);
   if (st != FP8BQ_OK) return st;
   if ((qt == nullptr) != (scales_t == nullptr)) return FP8BQ_ERR_INVALID_ARG;
@@ -262,7 +264,7 @@ int fp8bq_swiglu_quantize(const void* gu, int64_t M, int64_t F, int64_t ldgu, vo
   if (F % 128 != 0 || (qt != nullptr && M % 128 != 0)) return FP8BQ_ERR_SHAPE;
   if (M == 0 || F == 0) return FP8BQ_OK;
   if ((st = device_ok()) != FP8BQ_OK) return st;
-  return cuda_status(fp8bq::launch_swiglu_quant(gu, M, F, ldgu, h, q, scales, qt, scales_t, fmt,
+  return cuda_status(fp8bq::launch_swiglu_quant(gu, M, F, ldgu, h, q, scales, qt, scales_t, fmt, exact,
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -46,9 +46,10 @@ struct QuantJob {
 cudaError_t launch_quant_group(const QuantJob* jobs, int njobs, int fmt, cudaStream_t stream);
 
 // SwiGLU of [gate | up] fused with the quantization of its output h
-// (row groups, and token groups when qt != nullptr); h optionally stored.
+// (row groups, and token groups when qt != nullptr); h optionally stored;
+// exact: h rounded once from its exact value.
 cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* s_rows,
-                                void* qt, void* s_cols, int fmt, cudaStream_t stream);
+                                void* qt, void* s_cols, int fmt, bool exact, cudaStream_t stream);
 cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
                                  float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
                                  cudaStream_t stream);

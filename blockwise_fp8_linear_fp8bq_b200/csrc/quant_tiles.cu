@@ -102,21 +102,74 @@ __device__ __forceinline__ uint32_t rmsnorm_bf16x2(uint32_t x2, float2 rs2, floa
   return pack_bf16x2(h.x, h.y);
 }
 
-// h = silu(g) u = g u / (1 + e^-g) in fp32, rounded to bf16 (nearest, ties
-// to even; finite values).  The fast exponential and division keep the fp32
-// value within a few parts in 2^20 of the exact one, far inside the one-bf16-
-// ulp (2^-8) bound the result is specified to: the bf16 rounding hides them
-// except next to a rounding boundary.  For gate < -87, e^-g overflows and
-// h = +-0.
+// True when an fp32 value whose error bound is `ulp` ulps cannot be rounded
+// to bf16 with certainty: a rounding boundary (an fp32 whose low 16 bits are
+// 0x8000) lies within `ulp` of it, or it lies outside [2^-100, 2^127), where
+// its ulps stop being relative (or an intermediate may have overflowed).
+__device__ __forceinline__ bool bf16_undecided(float h, uint32_t ulp) {
+  const uint32_t mag = __float_as_uint(h) & 0x7FFFFFFFu;
+  const bool near = ((mag + (ulp - 0x8000u)) & 0xFFFFu) <= 2 * ulp;
+  const bool range = (mag - 0x0D800000u) >= (0x7F000000u - 0x0D800000u);
+  return near || range;
+}
+
+// h = silu(g) u = g u / (1 + e^-g) for one value the fast path left
+// undecided, rounded once to bf16 (nearest, ties to even).  First in fp32
+// with the accurate exponential (within 2 ulp, the documented bound of
+// expf), an exact add-then-round and the IEEE division: within
+// 2 (2 + 0.5 + 0.5) = 6 ulp of h for |g| <= 80; if that still leaves the
+// rounding open, in float64 in the order of the definition,
+// (g / (1 + e^-g)) u, rounded once from there.  Out of line: it runs for a
+// few values in a thousand.
+static __device__ __noinline__ uint32_t swiglu_slow_bf16(float g, float u) {
+  if (fabsf(g) <= 80.0f) {
+    const float h = __fdiv_rn(g * u, 1.0f + expf(-g));
+    if (!bf16_undecided(h, 8)) return pack_bf16x2(h, 0.0f) & 0xFFFFu;
+  }
+  const double gd = g;
+  const double v = gd / (1.0 + exp(-gd)) * static_cast<double>(u);
+  uint16_t r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(v));
+  return r;
+}
+
+// Ulps of the fast path's error bound (rounded up) and the gate magnitude
+// up to which it holds.
+constexpr uint32_t kSwiBoundUlp = 64;
+constexpr float kSwiGateMax = 16.0f;
+
+// h = silu(g) u = g u / (1 + e^-g) for two bf16 pairs, from the fp32 value
+// hf = g u / (1 + e^-g) with the fast exponential and division.
+//
+// Default (EXACT false): hf rounded to bf16 (nearest, ties to even; finite
+// values), within one bf16 ulp of the exact value: hf is within a few parts
+// in 2^20 of it, and the bf16 rounding hides that except next to a rounding
+// boundary.  For gate < -87, e^-g overflows and h = +-0.
+//
+// EXACT: each value rounded once to bf16 from the exact one.  g u is exact
+// (two 8-bit significands); the exponential is within 2 + floor(1.173 |g|)
+// ulp (the documented bound of __expf), the add within half an ulp, the
+// division within 2 ulp (__fdividef, divisor below 2^126), so hf is within
+// 2 (2 + 1.173 |g| + 2.5) < 48 ulp of h for |g| <= 16.  Its bf16 rounding is
+// h's unless bf16_undecided says otherwise; those values and |g| > 16 take
+// swiglu_slow_bf16.
+template <bool EXACT>
 __device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
-  float h[2];
+  float g[2], u[2], h[2];
+  bool slow[2];
 #pragma unroll
   for (int k = 0; k < 2; ++k) {
-    const float g = k ? bf16_hi(g2) : bf16_lo(g2);
-    const float u = k ? bf16_hi(u2) : bf16_lo(u2);
-    h[k] = __fdividef(g * u, 1.0f + __expf(-g));
+    g[k] = k ? bf16_hi(g2) : bf16_lo(g2);
+    u[k] = k ? bf16_hi(u2) : bf16_lo(u2);
+    h[k] = __fdividef(g[k] * u[k], 1.0f + __expf(-g[k]));
+    if constexpr (EXACT) slow[k] = bf16_undecided(h[k], kSwiBoundUlp) || !(fabsf(g[k]) <= kSwiGateMax);
   }
-  return pack_bf16x2(h[0], h[1]);  // round to nearest even
+  uint32_t r = pack_bf16x2(h[0], h[1]);  // round to nearest even
+  if constexpr (EXACT) {
+    if (slow[0]) r = (r & 0xFFFF0000u) | swiglu_slow_bf16(g[0], u[0]);
+    if (slow[1]) r = (r & 0x0000FFFFu) | (swiglu_slow_bf16(g[1], u[1]) << 16);
+  }
+  return r;
 }
 
 // Byte offset of 16-byte chunk c (0..15, 8 bf16 each) of tile row r: chunks
@@ -420,7 +473,7 @@ __device__ __forceinline__ void tile_block(const QParams& p, uint32_t base, int6
   if (warp == 0 && lane == 0) store_scale<FMT>(p.s_rows, (k0 / 128) * p.lds_m + m0 / 128, gs);
 }
 
-template <int FMT, bool ROWS, bool COLS, int G, bool SW, bool NORM>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW, bool NORM, bool EXACT>
 __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_constant__ QParams p) {
   static_assert(G == 128 || (G == 32 && FMT == kFmtUe8m0), "1x32 groups use UE8M0 scales");
   using C = QCfg<SW>;
@@ -539,8 +592,8 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
           if constexpr (SW) {
             const uint4 g = ld_shared_v4(base + off);
             const uint4 u = ld_shared_v4(base + kQStage + off);
-            hv[i] = make_uint4(swiglu_bf16x2(g.x, u.x), swiglu_bf16x2(g.y, u.y), swiglu_bf16x2(g.z, u.z),
-                               swiglu_bf16x2(g.w, u.w));
+            hv[i] = make_uint4(swiglu_bf16x2<EXACT>(g.x, u.x), swiglu_bf16x2<EXACT>(g.y, u.y),
+                               swiglu_bf16x2<EXACT>(g.z, u.z), swiglu_bf16x2<EXACT>(g.w, u.w));
           } else {
             const float2 rs2 = make_float2(rsv[i], rsv[i]);
             const uint4 x = ld_shared_v4(base + off);
@@ -685,9 +738,9 @@ bool encode_x(CUtensorMap* map, const void* x, int64_t rows, int64_t cols, int64
   return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool ROWS, bool COLS, int G, bool SW = false, bool NORM = false>
+template <int FMT, bool ROWS, bool COLS, int G, bool SW = false, bool NORM = false, bool EXACT = false>
 cudaError_t launch_tiles(const QParams& prm, cudaStream_t stream) {
-  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G, SW, NORM>;
+  auto kern = quant_tile_kernel<FMT, ROWS, COLS, G, SW, NORM, EXACT>;
   constexpr uint32_t kQSmem = QCfg<SW>::kSmem;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -825,8 +878,9 @@ cudaError_t launch_quant_tiles(const void* x, int64_t M, int64_t K, int64_t ldx,
 // [gate | up] -> h = silu(gate) * up (BF16, optionally stored to h [M, F]),
 // quantized as quantize_act (q, s_rows) and, when qt != nullptr, as
 // quantize_act_t (qt, s_cols).  F % 128 == 0; M % 128 == 0 when qt is set.
+// exact: h rounded once from the exact value (swiglu_bf16x2<true>).
 cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ldgu, void* h, void* q, void* s_rows,
-                                void* qt, void* s_cols, int fmt, cudaStream_t stream) {
+                                void* qt, void* s_cols, int fmt, bool exact, cudaStream_t stream) {
   QParams prm;
   std::memset(&prm, 0, sizeof(prm));
   if (!encode_x(&prm.tmX, gu, M, 2 * F, ldgu)) return cudaErrorInvalidValue;
@@ -852,6 +906,13 @@ cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ld
   prm.status = status;
   prm.limit_ns = 2000000000ull;
   const bool cols = qt != nullptr;
+  if (exact) {
+    if (fmt == kFmtFp32)
+      return cols ? launch_tiles<kFmtFp32, true, true, 128, true, false, true>(prm, stream)
+                  : launch_tiles<kFmtFp32, true, false, 128, true, false, true>(prm, stream);
+    return cols ? launch_tiles<kFmtUe8m0, true, true, 128, true, false, true>(prm, stream)
+                : launch_tiles<kFmtUe8m0, true, false, 128, true, false, true>(prm, stream);
+  }
   if (fmt == kFmtFp32)
     return cols ? launch_tiles<kFmtFp32, true, true, 128, true>(prm, stream)
                 : launch_tiles<kFmtFp32, true, false, 128, true>(prm, stream);

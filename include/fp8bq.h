@@ -74,6 +74,9 @@ typedef enum { FP8BQ_E4M3 = 0, FP8BQ_BF16 = 1 } fp8bq_dtype;
 /* fp8bq_gemm flags */
 #define FP8BQ_GEMM_ACCUMULATE_F32 1u /* D is FP32 and D += A B^T */
 
+/* fp8bq_swiglu_quantize: OR into fmt to round h once from its exact value */
+#define FP8BQ_SWIGLU_EXACT 0x100
+
 /*
  * One GEMM operand, seen as a logical matrix [rows, C] whose second index runs
  * over the contraction C.
@@ -168,13 +171,19 @@ int fp8bq_quantize_act_dual(const void* x, int64_t M, int64_t K, int64_t ldx, vo
  *   h         optional BF16 [M, F] (ld F): h = silu(gate) * up =
  *             gate * up / (1 + e^-gate) in FP32, rounded to BF16 (nearest,
  *             ties to even); may be NULL.  Within one BF16 ulp of the exact
- *             value.
+ *             value (while gate * up stays below the FP32 maximum); with
+ *             FP8BQ_SWIGLU_EXACT in fmt, the exact value rounded
+ *             once to BF16 (nearest, ties to even): the FP32 value where its
+ *             error bound decides the rounding, float64 (the definition's
+ *             order, (gate / (1 + e^-gate)) * up) for the rest; ~60% more
+ *             time.
  *   q, scales h quantized as fp8bq_quantize_act (1x128 groups along F) of
  *             exactly that BF16 h: E4M3 [M, F] (ld F), scales
  *             [F/128][fp8bq_row_scale_ld(M)].
  *   qt, scales_t  optional (both or neither): h quantized as
  *             fp8bq_quantize_act_t: [F, M] (ld M), [M/128][fp8bq_row_scale_ld(F)].
- *   fmt       FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0.
+ *   fmt       FP8BQ_SCALE_FP32 or FP8BQ_SCALE_UE8M0, optionally OR
+ *             FP8BQ_SWIGLU_EXACT.
  * Errors: ERR_INVALID_ARG (null gu, q or scales; only one of qt, scales_t;
  * bad fmt), ERR_SHAPE (F % 128 != 0; M % 128 != 0 with qt; ldgu < 2F),
  * ERR_ALIGN (as fp8bq_quantize_act, and h, qt, scales_t 16-B aligned).

@@ -240,6 +240,9 @@ def test_swiglu_quantize_argument_checks(L):
     assert g(q=None) == INVALID
     assert g(qt=P) == INVALID                 # qt without scales_t
     assert g(fmt=3) == INVALID
+    assert g(fmt=0x100 | 3) == INVALID        # the exact flag with a bad format
+    assert g(fmt=0x100 | 1, gu=None) == INVALID
+    assert g(fmt=0x100 | 1, M=0) == OK        # the exact flag is accepted
     assert g(F=100, ld=200) == SHAPE          # F % 128
     assert g(ld=128) == SHAPE                 # ldgu < 2F
     assert g(M=100, qt=P, st=P) == SHAPE      # tokens % 128 with transposed codes
