@@ -814,6 +814,13 @@ def case_launchers(step, fp):
                                          lambda it=it: fp.rmsnorm_quantize(
                                              it["x"], it["gamma"], 1e-6, f,
                                              out=(it["qx"], it["sx"], it["qxt"], it["sxt"], None, it["rstd"])))
+            # the same with h rounded once from its exact value (rstd in float64)
+            it["rstd64"] = torch.empty(M, dtype=torch.float64, device=it["x"].device)
+            out[f"quant_rmsnorm_exact:{n}"] = ("quant", M * K * 4 + ((K // 128) * M + (M // 128) * K) * sb + 8 * M
+                                               + 2 * K, lambda it=it: fp.rmsnorm_quantize(
+                                                   it["x"], it["gamma"], 1e-6, f, exact=True,
+                                                   out=(it["qx"], it["sx"], it["qxt"], it["sxt"], None,
+                                                        it["rstd64"])))
         # fused quantize-on-load: BF16 A quantized inside the GEMM
         out[f"gemm_fwd_fused:{n}"] = ("gemm", lin.flops, lambda it=it: fp.gemm(
             fp.bf16_operand(it["x"], f), fp.block_operand(it["qw"], it["sw"], f), it["y"], workspace=step.ws))

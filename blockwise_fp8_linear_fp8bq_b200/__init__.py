@@ -109,6 +109,9 @@ def lib():
         L.fp8bq_swiglu_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, i32, vp]
         L.fp8bq_rmsnorm_quantize.restype = i32
         L.fp8bq_rmsnorm_quantize.argtypes = [vp, i64, i64, i64, vp, ctypes.c_float, vp, vp, vp, vp, vp, vp, i32, vp]
+        L.fp8bq_rmsnorm_quantize_exact.restype = i32
+        L.fp8bq_rmsnorm_quantize_exact.argtypes = [vp, i64, i64, i64, vp, ctypes.c_double, vp, vp, vp, vp, vp, vp,
+                                                   i32, vp]
         L.fp8bq_quantize_act_dual_mx.restype = i32
         L.fp8bq_quantize_act_dual_mx.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp]
         L.fp8bq_quantize_group.restype = i32
@@ -245,12 +248,13 @@ def swiglu_quantize(gu: torch.Tensor, fmt: int = SCALE_FP32, transposed: bool = 
 
 
 def rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, fmt: int = SCALE_FP32,
-                     transposed: bool = True, keep_h: bool = False, out=None):
+                     transposed: bool = True, keep_h: bool = False, out=None, exact: bool = False):
     """x bf16 [M, K], gamma bf16 [K] -> (q, s, qt, st, h, rstd): h = x * rstd * gamma in
     BF16 (rstd = 1 / sqrt(mean(x^2) + eps), fp32 [M]) quantized as quantize_act (q, s)
     and, with transposed, quantize_act_t (qt, st); h is returned when keep_h (else
     None), qt/st are None without transposed.  `out` may pass (q, s, qt, st, h, rstd)
-    to write into."""
+    to write into.  exact: fp8bq_rmsnorm_quantize_exact (rstd float64 [M], h rounded
+    once from its exact value)."""
     _check_bf16(x, "x")
     M, K = x.shape
     if (not gamma.is_cuda or gamma.dtype != torch.bfloat16 or gamma.numel() != K or not gamma.is_contiguous()
@@ -262,11 +266,12 @@ def rmsnorm_quantize(x: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-6, fm
     qt = _out(o[2], (K, M), torch.float8_e4m3fn, x.device) if transposed else None
     st = _out(o[3], (M // 128, row_scale_ld(K)), _scale_dtype(fmt), x.device) if transposed else None
     h = _out(o[4], (M, K), torch.bfloat16, x.device) if keep_h else None
-    rstd = _out(o[5], (M,), torch.float32, x.device)
+    rstd = _out(o[5], (M,), torch.float64 if exact else torch.float32, x.device)
     ptr = lambda t: t.data_ptr() if t is not None else None
-    rc = lib().fp8bq_rmsnorm_quantize(x.data_ptr(), M, K, x.stride(0), gamma.data_ptr(), float(eps), rstd.data_ptr(),
-                                      ptr(h), q.data_ptr(), s.data_ptr(), ptr(qt), ptr(st), fmt, _stream(x))
-    _raise(rc, "fp8bq_rmsnorm_quantize")
+    call = lib().fp8bq_rmsnorm_quantize_exact if exact else lib().fp8bq_rmsnorm_quantize
+    rc = call(x.data_ptr(), M, K, x.stride(0), gamma.data_ptr(), float(eps), rstd.data_ptr(), ptr(h), q.data_ptr(),
+              s.data_ptr(), ptr(qt), ptr(st), fmt, _stream(x))
+    _raise(rc, "fp8bq_rmsnorm_quantize_exact" if exact else "fp8bq_rmsnorm_quantize")
     return q, s, qt, st, h, rstd
 
 

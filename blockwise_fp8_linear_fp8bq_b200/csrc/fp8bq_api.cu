@@ -286,6 +286,24 @@ int fp8bq_rmsnorm_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, con
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int fp8bq_rmsnorm_quantize_exact(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, double eps,
+                                 double* rstd, void* h, void* q, void* scales, void* qt, void* scales_t, int fmt,
+                                 fp8bq_stream_t stream) {
+  int st = check_quant_args(x, M, K, ldx, q, scales, fmt);
+  if (st != FP8BQ_OK) return st;
+  if (gamma == nullptr || rstd == nullptr) return FP8BQ_ERR_INVALID_ARG;
+  if (!(eps >= 0.0) || eps > 1.0e300) return FP8BQ_ERR_INVALID_ARG;  // finite, not negative
+  if ((qt == nullptr) != (scales_t == nullptr)) return FP8BQ_ERR_INVALID_ARG;
+  if (!aligned16(gamma) || (reinterpret_cast<uintptr_t>(rstd) & 7u) != 0) return FP8BQ_ERR_ALIGN;
+  if (qt != nullptr && (!aligned16(qt) || !aligned16(scales_t))) return FP8BQ_ERR_ALIGN;
+  if (h != nullptr && !aligned16(h)) return FP8BQ_ERR_ALIGN;
+  if (K % 128 != 0 || (qt != nullptr && M % 128 != 0)) return FP8BQ_ERR_SHAPE;
+  if (M == 0 || K == 0) return FP8BQ_OK;
+  if ((st = device_ok()) != FP8BQ_OK) return st;
+  return cuda_status(fp8bq::launch_rmsnorm_quant_exact(x, M, K, ldx, gamma, eps, rstd, h, q, scales, qt, scales_t,
+                                                       fmt, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int fp8bq_quantize_weight(const void* w, int64_t N, int64_t K, int64_t ldw, void* q, void* scales,
                           int fmt, fp8bq_stream_t stream) {
   int st = check_quant_args(w, N, K, ldw, q, scales, fmt);

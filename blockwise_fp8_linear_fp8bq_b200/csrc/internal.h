@@ -53,6 +53,10 @@ cudaError_t launch_swiglu_quant(const void* gu, int64_t M, int64_t F, int64_t ld
 cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
                                  float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
                                  cudaStream_t stream);
+// The same with h rounded once from its exact value; rstd64 [M] in float64.
+cudaError_t launch_rmsnorm_quant_exact(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                       double eps, double* rstd64, void* h, void* q, void* s_rows, void* qt,
+                                       void* s_cols, int fmt, cudaStream_t stream);
 
 // Driver entry point of cuTensorMapEncodeTiled (nullptr if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();

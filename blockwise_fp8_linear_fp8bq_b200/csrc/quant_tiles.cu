@@ -75,6 +75,7 @@ struct QParams {
   int64_t ldh;
   // RMSNorm producer: X is h = x * rstd[row] * gamma[col]
   const float* rstd;       // [M]
+  const double* rstd64;    // [M], the exact RMSNorm's float64 row statistic
   const uint16_t* gamma;   // BF16 [K]
 };
 
@@ -169,6 +170,43 @@ __device__ __forceinline__ uint32_t swiglu_bf16x2(uint32_t g2, uint32_t u2) {
     if (slow[0]) r = (r & 0xFFFF0000u) | swiglu_slow_bf16(g[0], u[0]);
     if (slow[1]) r = (r & 0x0000FFFFu) | (swiglu_slow_bf16(g[1], u[1]) << 16);
   }
+  return r;
+}
+
+// RMSNorm rounded once from the exact value h = x rstd gamma, given rstd in
+// float64 (rs64) and rs = its fp32 rounding.  With rs, t = x rs and hf =
+// t gamma all normal fp32 values, hf is within 2^-24 (rs) + 2 x 2^-24 (the
+// two products' roundings) of h, relative, i.e. within 3 ulp (plus the
+// float64 rstd's own error, below 2^-33 for any K): its bf16 rounding is h's
+// unless bf16_undecided(hf, 8) says otherwise.  Those values, and the values
+// of a row whose rs is not a normal fp32 (row_slow) or whose t is not one,
+// are evaluated in float64 in the definition's order, (x rstd) gamma, and
+// rounded once.
+constexpr uint32_t kNormBoundUlp = 8;
+
+static __device__ __noinline__ uint32_t rmsnorm_f64_bf16(float x, double rs64, float g) {
+  const double v = static_cast<double>(x) * rs64 * static_cast<double>(g);
+  uint16_t r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(v));
+  return r;
+}
+
+// |v| outside [2^-126, 2^127): not a normal fp32 (or near overflow).
+__device__ __forceinline__ bool f32_not_normal(float v) {
+  const uint32_t mag = __float_as_uint(v) & 0x7FFFFFFFu;
+  return (mag - 0x00800000u) >= (0x7F000000u - 0x00800000u);
+}
+
+__device__ __forceinline__ uint32_t rmsnorm_exact_bf16x2(uint32_t x2, float2 rs2, float2 g, double rs64,
+                                                         bool row_slow) {
+  const float2 xx = make_float2(bf16_lo(x2), bf16_hi(x2));
+  const float2 t = __fmul2_rn(xx, rs2);
+  const float2 h = __fmul2_rn(t, g);
+  uint32_t r = pack_bf16x2(h.x, h.y);
+  if (row_slow || f32_not_normal(t.x) || bf16_undecided(h.x, kNormBoundUlp))
+    r = (r & 0xFFFF0000u) | rmsnorm_f64_bf16(xx.x, rs64, g.x);
+  if (row_slow || f32_not_normal(t.y) || bf16_undecided(h.y, kNormBoundUlp))
+    r = (r & 0x0000FFFFu) | (rmsnorm_f64_bf16(xx.y, rs64, g.y) << 16);
   return r;
 }
 
@@ -546,6 +584,7 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
     // the tile at hand (loaded one tile ahead, off the critical path)
     uint4 ng = make_uint4(0, 0, 0, 0);
     float nrs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    double nrs64[4] = {0.0, 0.0, 0.0, 0.0};  // exact RMSNorm: rstd in float64
     auto norm_load = [&](int tile) {
       if (tile >= p.num_tiles) return;
       int64_t tm0, tk0;
@@ -554,7 +593,12 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int64_t r = tm0 + 8 * warp + 2 * i + (lane >> 4);
-        nrs[i] = r < p.M ? __ldg(p.rstd + r) : 0.0f;
+        if constexpr (EXACT) {
+          nrs64[i] = r < p.M ? __ldg(p.rstd64 + r) : 0.0;
+          nrs[i] = __double2float_rn(nrs64[i]);
+        } else {
+          nrs[i] = r < p.M ? __ldg(p.rstd + r) : 0.0f;
+        }
       }
     };
     if constexpr (NORM) norm_load(blockIdx.x);
@@ -576,13 +620,17 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
         uint4 hv[4];
         float2 g0, g1, g2, g3;
         float rsv[4];
+        double rsv64[4];
         if constexpr (NORM) {
           g0 = make_float2(bf16_lo(ng.x), bf16_hi(ng.x));
           g1 = make_float2(bf16_lo(ng.y), bf16_hi(ng.y));
           g2 = make_float2(bf16_lo(ng.z), bf16_hi(ng.z));
           g3 = make_float2(bf16_lo(ng.w), bf16_hi(ng.w));
 #pragma unroll
-          for (int i = 0; i < 4; ++i) rsv[i] = nrs[i];
+          for (int i = 0; i < 4; ++i) {
+            rsv[i] = nrs[i];
+            rsv64[i] = nrs64[i];
+          }
           norm_load(tile + gridDim.x);
         }
 #pragma unroll
@@ -597,8 +645,15 @@ __global__ void __launch_bounds__(kQThreads, 1) quant_tile_kernel(const __grid_c
           } else {
             const float2 rs2 = make_float2(rsv[i], rsv[i]);
             const uint4 x = ld_shared_v4(base + off);
-            hv[i] = make_uint4(rmsnorm_bf16x2(x.x, rs2, g0), rmsnorm_bf16x2(x.y, rs2, g1),
-                               rmsnorm_bf16x2(x.z, rs2, g2), rmsnorm_bf16x2(x.w, rs2, g3));
+            if constexpr (EXACT) {
+              const bool row_slow = f32_not_normal(rsv[i]);
+              hv[i] = make_uint4(rmsnorm_exact_bf16x2(x.x, rs2, g0, rsv64[i], row_slow),
+                                 rmsnorm_exact_bf16x2(x.y, rs2, g1, rsv64[i], row_slow),
+                                 rmsnorm_exact_bf16x2(x.z, rs2, g2, rsv64[i], row_slow),
+                                 rmsnorm_exact_bf16x2(x.w, rs2, g3, rsv64[i], row_slow));
+            } else
+              hv[i] = make_uint4(rmsnorm_bf16x2(x.x, rs2, g0), rmsnorm_bf16x2(x.y, rs2, g1),
+                                 rmsnorm_bf16x2(x.z, rs2, g2), rmsnorm_bf16x2(x.w, rs2, g3));
           }
           st_shared_v4(base + off, hv[i].x, hv[i].y, hv[i].z, hv[i].w);
           if (p.h != nullptr && m0 + r < p.M)
@@ -947,21 +1002,36 @@ __global__ void __launch_bounds__(256) rstd_kernel(const uint16_t* __restrict__ 
   if (lane == 0) rstd[r] = __fdiv_rn(1.0f, __fsqrt_rn(__fdiv_rn(acc, static_cast<float>(K)) + eps));
 }
 
-}  // namespace
+// The same statistic in float64 (each x^2 exact, the sum, the mean, eps, the
+// square root and the reciprocal in IEEE double): the exact RMSNorm's rstd.
+__global__ void __launch_bounds__(256) rstd64_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t K,
+                                                     int64_t ldx, double eps, double* __restrict__ rstd64) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= M) return;
+  const uint16_t* row = x + r * ldx;
+  double acc = 0.0;
+#pragma unroll 4
+  for (int64_t k = 8 * lane; k < K; k += 256) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(row + k));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double a = bf16_lo(w[i]), b = bf16_hi(w[i]);
+      acc = fma(a, a, acc);
+      acc = fma(b, b, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) rstd64[r] = 1.0 / sqrt(acc / static_cast<double>(K) + eps);
+}
 
-// RMSNorm fused with the quantization of its output: x BF16 [M, K] ->
-// rstd [M] (fp32) -> h = x * rstd * gamma (BF16, optionally stored to h
-// [M, K]), quantized as quantize_act (q, s_rows) and, when qt != nullptr, as
-// quantize_act_t (qt, s_cols).  K % 128 == 0; M % 128 == 0 when qt is set.
-cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
-                                 float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
-                                 cudaStream_t stream) {
-  const int64_t blocks = (M + 7) / 8;
-  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
-  rstd_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), M, K, ldx, eps,
-                                                                 rstd);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+// The RMSNorm tile pass, after the row statistics: rstd (fp32) for the
+// default rounding, or rstd64 (float64, rstd == nullptr) for the exact one.
+cudaError_t launch_norm_tiles(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, const float* rstd,
+                              const double* rstd64, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
+                              cudaStream_t stream) {
   QParams prm;
   std::memset(&prm, 0, sizeof(prm));
   if (!encode_x(&prm.tmX, x, M, K, ldx)) return cudaErrorInvalidValue;
@@ -981,18 +1051,59 @@ cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ld
   prm.h = static_cast<uint16_t*>(h);
   prm.ldh = K;
   prm.rstd = rstd;
+  prm.rstd64 = rstd64;
   prm.gamma = static_cast<const uint16_t*>(gamma);
   int* status = nullptr;
-  e = device_status_word(&status);
+  const cudaError_t e = device_status_word(&status);
   if (e != cudaSuccess) return e;
   prm.status = status;
   prm.limit_ns = 2000000000ull;
   const bool cols = qt != nullptr;
+  if (rstd64 != nullptr) {
+    if (fmt == kFmtFp32)
+      return cols ? launch_tiles<kFmtFp32, true, true, 128, false, true, true>(prm, stream)
+                  : launch_tiles<kFmtFp32, true, false, 128, false, true, true>(prm, stream);
+    return cols ? launch_tiles<kFmtUe8m0, true, true, 128, false, true, true>(prm, stream)
+                : launch_tiles<kFmtUe8m0, true, false, 128, false, true, true>(prm, stream);
+  }
   if (fmt == kFmtFp32)
     return cols ? launch_tiles<kFmtFp32, true, true, 128, false, true>(prm, stream)
                 : launch_tiles<kFmtFp32, true, false, 128, false, true>(prm, stream);
   return cols ? launch_tiles<kFmtUe8m0, true, true, 128, false, true>(prm, stream)
               : launch_tiles<kFmtUe8m0, true, false, 128, false, true>(prm, stream);
+}
+
+}  // namespace
+
+// RMSNorm fused with the quantization of its output: x BF16 [M, K] ->
+// rstd [M] (fp32) -> h = x * rstd * gamma (BF16, optionally stored to h
+// [M, K]), quantized as quantize_act (q, s_rows) and, when qt != nullptr, as
+// quantize_act_t (qt, s_cols).  K % 128 == 0; M % 128 == 0 when qt is set.
+cudaError_t launch_rmsnorm_quant(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, float eps,
+                                 float* rstd, void* h, void* q, void* s_rows, void* qt, void* s_cols, int fmt,
+                                 cudaStream_t stream) {
+  const int64_t blocks = (M + 7) / 8;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  rstd_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), M, K, ldx, eps,
+                                                                 rstd);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_norm_tiles(x, M, K, ldx, gamma, rstd, nullptr, h, q, s_rows, qt, s_cols, fmt, stream);
+}
+
+// The same with h rounded once from its exact value: rstd in float64
+// (rstd64 [M], written), the fp32 products where their error bound decides
+// the bf16 rounding, float64 for the rest (rmsnorm_exact_bf16x2).
+cudaError_t launch_rmsnorm_quant_exact(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma,
+                                       double eps, double* rstd64, void* h, void* q, void* s_rows, void* qt,
+                                       void* s_cols, int fmt, cudaStream_t stream) {
+  const int64_t blocks = (M + 7) / 8;
+  if (blocks > INT32_MAX) return cudaErrorInvalidValue;
+  rstd64_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const uint16_t*>(x), M, K, ldx,
+                                                                   eps, rstd64);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_norm_tiles(x, M, K, ldx, gamma, nullptr, rstd64, h, q, s_rows, qt, s_cols, fmt, stream);
 }
 
 }  // namespace fp8bq

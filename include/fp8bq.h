@@ -223,6 +223,24 @@ int fp8bq_rmsnorm_quantize(const void* x, int64_t M, int64_t K, int64_t ldx, con
                            fp8bq_stream_t stream);
 
 /*
+ * fp8bq_rmsnorm_quantize with h rounded once from its exact value, so that
+ * h, codes and scales equal the float64 definition's bit for bit.
+ *   eps       added to the mean square (finite, >= 0), in double.
+ *   rstd      float64 [M] (8-byte aligned), written: 1 / sqrt(mean_k x[r,k]^2
+ *             + eps) in IEEE double (each square exact, the sum in double).
+ *   h         optional BF16 [M, K] (ld K): x * rstd * gamma rounded once to
+ *             BF16 (nearest, ties to even) from the exact product: the FP32
+ *             products (of x, rstd rounded to FP32, and gamma) where their
+ *             error bound (3 ulp) keeps every BF16 rounding boundary out of
+ *             reach, float64 ((x * rstd) * gamma) for the rest.
+ *   the other arguments and the errors as fp8bq_rmsnorm_quantize
+ *   (ERR_ALIGN for an rstd not 8-byte aligned).
+ */
+int fp8bq_rmsnorm_quantize_exact(const void* x, int64_t M, int64_t K, int64_t ldx, const void* gamma, double eps,
+                                 double* rstd, void* h, void* q, void* scales, void* qt, void* scales_t, int fmt,
+                                 fp8bq_stream_t stream);
+
+/*
  * MX-block quantization (1x32 groups, UE8M0 scales): the other reading of
  * "MXFP8 on Blackwell" ("方法"), with the OCP Microscaling format's 32-value
  * blocks in place of the 1x128 groups.  Same definitions as the calls above

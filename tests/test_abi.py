@@ -273,6 +273,24 @@ def test_rmsnorm_quantize_argument_checks(L):
     assert g(M=0) == OK                       # empty: no launch
 
 
+def test_rmsnorm_quantize_exact_argument_checks(L):
+    f = L.fp8bq_rmsnorm_quantize_exact
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p, ctypes.c_double,
+                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                  ctypes.c_int, ctypes.c_void_p]
+    g = lambda x=P, M=128, K=256, ld=256, gamma=P, eps=1e-6, rstd=P, h=None, q=P, s=P, qt=None, st=None, fmt=1: f(
+        x, M, K, ld, gamma, eps, rstd, h, q, s, qt, st, fmt, None)
+    assert g(x=None) == INVALID
+    assert g(rstd=None) == INVALID
+    assert g(eps=-1.0) == INVALID
+    assert g(eps=float("inf")) == INVALID
+    assert g(fmt=2) == INVALID
+    assert g(K=200, ld=200) == SHAPE          # K % 128
+    assert g(rstd=P + 4) == ALIGN             # float64 rstd: 8-byte aligned
+    assert g(M=0) == OK                       # empty: no launch
+
+
 def test_quantize_group_argument_checks(L):
     import blockwise_fp8_linear_fp8bq_b200 as fp
     f = L.fp8bq_quantize_group
