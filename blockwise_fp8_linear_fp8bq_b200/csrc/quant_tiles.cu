@@ -16,6 +16,12 @@
 // consumer warps quantize out of shared memory and store codes and scales
 // straight from registers.  Every wait is bounded (status word, as in the
 // GEMM).
+//
+// The producer ops feed the same kernel: SwiGLU of a [gate | up] tile pair
+// and RMSNorm of an X tile (with its row statistics from rstd_kernel), each
+// warp computing the BF16 h of the rows it quantizes.  Their EXACT variants
+// round h once from its exact value: FP32 where a proven error bound decides
+// the BF16 rounding, float64 for the few values it leaves open.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
