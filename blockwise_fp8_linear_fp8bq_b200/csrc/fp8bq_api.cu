@@ -3,6 +3,7 @@
 // memory or synchronizes, except fp8bq_check().
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -292,7 +293,7 @@ int fp8bq_rmsnorm_quantize_exact(const void* x, int64_t M, int64_t K, int64_t ld
   int st = check_quant_args(x, M, K, ldx, q, scales, fmt);
   if (st != FP8BQ_OK) return st;
   if (gamma == nullptr || rstd == nullptr) return FP8BQ_ERR_INVALID_ARG;
-  if (!(eps >= 0.0) || eps > 1.0e300) return FP8BQ_ERR_INVALID_ARG;  // finite, not negative
+  if (!(eps >= 0.0) || !std::isfinite(eps)) return FP8BQ_ERR_INVALID_ARG;  // finite, not negative
   if ((qt == nullptr) != (scales_t == nullptr)) return FP8BQ_ERR_INVALID_ARG;
   if (!aligned16(gamma) || (reinterpret_cast<uintptr_t>(rstd) & 7u) != 0) return FP8BQ_ERR_ALIGN;
   if (qt != nullptr && (!aligned16(qt) || !aligned16(scales_t))) return FP8BQ_ERR_ALIGN;
