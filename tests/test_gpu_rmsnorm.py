@@ -95,3 +95,19 @@ def test_rmsnorm_quantize_full_size(fmt, exact):
     x = synth.activations_bf16(16384, synth.HIDDEN, seed=85, device="cuda")
     rows = np.sort(np.random.default_rng(86).choice(16384, 64, replace=False))
     check(x, gamma_of(synth.HIDDEN, 87), fmt, True, sample_rows=rows, exact=exact)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_rmsnorm_exact_stress(fmt):
+    """Exact mode on rows whose magnitudes differ by up to 2^80 and whose
+    values spread over 40 binades within a row, with gamma over 20 binades;
+    h bit for bit against the oracle."""
+    M, K = 256, 1024
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(88)
+    row_scale = torch.exp2(torch.rand(M, 1, generator=gen, device="cuda") * 80.0 - 40.0)
+    mag = torch.exp2(torch.rand(M, K, generator=gen, device="cuda") * 40.0 - 20.0)
+    sign = torch.where(torch.rand(M, K, generator=gen, device="cuda") < 0.5, -1.0, 1.0)
+    x = (row_scale * mag * sign).to(torch.bfloat16)
+    gamma = (torch.exp2(torch.rand(K, generator=gen, device="cuda") * 20.0 - 10.0)).to(torch.bfloat16)
+    check(x, gamma, fmt, True, exact=True)

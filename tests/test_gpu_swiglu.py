@@ -90,3 +90,19 @@ def test_swiglu_quantize_ragged_rows(fmt, exact):
 def test_swiglu_quantize_full_size(fmt, exact):
     """The down projection's input of the layer: [16384, 2 x 6144] -> h [16384, 6144]."""
     check(gate_up(16384, synth.MLP, 73), fmt, True, exact)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_swiglu_exact_stress(fmt):
+    """Exact mode across its fast path's whole range: gates uniform in
+    [-16, 16] (where the fast exponential's error bound is largest) and up
+    values spread over 120 binades, both signs; h bit for bit against the
+    oracle."""
+    M, F = 512, 2048
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(74)
+    g = (torch.rand(M, F, generator=gen, device="cuda") * 32.0 - 16.0).to(torch.bfloat16)
+    mag = torch.exp2(torch.rand(M, F, generator=gen, device="cuda") * 120.0 - 60.0)
+    sign = torch.where(torch.rand(M, F, generator=gen, device="cuda") < 0.5, -1.0, 1.0)
+    u = (mag * sign).to(torch.bfloat16)
+    check(torch.cat([g, u], dim=1).contiguous(), fmt, True, True)
