@@ -123,7 +123,7 @@ __device__ __forceinline__ bool bf16_undecided(float h, uint32_t ulp) {
 // h = silu(g) u = g u / (1 + e^-g) for one value the fast path left
 // undecided, rounded once to bf16 (nearest, ties to even).  First in fp32
 // with the accurate exponential (within 2 ulp, the documented bound of
-// expf), an exact add-then-round and the IEEE division: within
+// expf), the add (half an ulp) and the IEEE division (half an ulp): within
 // 2 (2 + 0.5 + 0.5) = 6 ulp of h for |g| <= 80; if that still leaves the
 // rounding open, in float64 in the order of the definition,
 // (g / (1 + e^-g)) u, rounded once from there.  Out of line: it runs for a
